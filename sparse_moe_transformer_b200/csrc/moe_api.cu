@@ -1,0 +1,647 @@
+// moe_api.cu -- host runtime behind include/moe.h: handle, owned weight copies,
+// workspace, second stream for the shared expert, TMA descriptors, error words.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "layer.h"
+
+using namespace moe;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+moe_status fail(moe_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+#define CUDA_TRY(expr)                                                                   \
+    do {                                                                                 \
+        cudaError_t e_ = (expr);                                                         \
+        if (e_ != cudaSuccess)                                                           \
+            return fail(e_ == cudaErrorMemoryAllocation ? MOE_ERR_OOM : MOE_ERR_CUDA,    \
+                        "%s: %s (%s:%d)", #expr, cudaGetErrorString(e_), __FILE__, __LINE__); \
+    } while (0)
+
+// Restores the caller's current device on scope exit.
+struct DeviceGuard {
+    int prev = -1;
+    explicit DeviceGuard(int dev) {
+        cudaGetDevice(&prev);
+        if (prev != dev) cudaSetDevice(dev);
+    }
+    ~DeviceGuard() {
+        int cur = -1;
+        cudaGetDevice(&cur);
+        if (prev >= 0 && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2D bf16 tensor map over a row-major [rows][cols] matrix: boxes of 64 columns
+// (one 128-byte swizzle row) by box_rows rows, 128-byte swizzle, zero fill.
+moe_status make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    if ((reinterpret_cast<uintptr_t>(base) & 15) || (cols * 2) % 16)
+        return fail(MOE_ERR_INVALID_ARG, "tensor map base/stride not 16-byte aligned");
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return MOE_OK;
+}
+
+constexpr int kRouteBlock = 16;      // tokens per router CTA / permutation block
+constexpr int kNarrow = 32, kWide = 256;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace
+
+struct moe_layer {
+    moe_config cfg;
+    Dims d;
+    int device = 0;
+    int dtype = 1;
+    size_t esz = 2;
+    bool tc_ok = false;
+    int num_sms = 148;
+    // owned weight copies
+    void *w_router = nullptr, *w_gate = nullptr, *w_up = nullptr, *w_down = nullptr;
+    void *ws_gate = nullptr, *ws_up = nullptr, *ws_down = nullptr, *rms_w = nullptr;
+    // workspace
+    int max_T = 0;
+    int max_units = 0;
+    char* ws = nullptr;
+    RouteBufs rb{};
+    void *x_norm = nullptr, *xp = nullptr, *hbuf = nullptr, *obuf = nullptr;
+    void *hs = nullptr, *sbuf = nullptr;
+    void *x_stage = nullptr, *r_stage = nullptr, *y_stage = nullptr;
+    int32_t *sync_routed = nullptr, *sync_shared = nullptr;
+    TcMaps routed_maps{}, shared_maps{};
+    // status words
+    int* err_dev = nullptr;
+    int* err_host = nullptr;
+    int* err_host_dev = nullptr;
+    // streams
+    cudaStream_t s2 = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+    // options
+    uint64_t wait_limit_ns = 1000000000ull;
+    int inject_stuck = 0, shared_stream = 1, fuse = 1, force_simt = 0, timing = 0;
+    int last_T = 0;
+    // kernel statistics
+    struct Pending { int cls; cudaEvent_t a, b; };
+    std::vector<cudaEvent_t> ev_pool;
+    std::vector<Pending> pending;
+    double k_ms[MOE_KERNEL_CLASSES] = {};
+    int64_t k_launches[MOE_KERNEL_CLASSES] = {};
+
+    DeviceStatus status() const { return DeviceStatus{err_dev, err_host_dev}; }
+};
+
+namespace {
+
+moe_status copy_weight(void** dst, const void* src, size_t bytes) {
+    if (!bytes) return MOE_OK;
+    CUDA_TRY(cudaMalloc(dst, bytes));
+    CUDA_TRY(cudaMemcpy(*dst, src, bytes, cudaMemcpyDeviceToDevice));
+    return MOE_OK;
+}
+
+void free_workspace(moe_layer* h) {
+    if (h->ws) cudaFree(h->ws);
+    h->ws = nullptr;
+    h->max_T = 0;
+}
+
+moe_status pending_device_error(moe_layer* h) {
+    int code = h->err_host ? *(volatile int*)h->err_host : 0;
+    if (code == MOE_ERR_TIMEOUT)
+        return fail(MOE_ERR_TIMEOUT, "a bounded device-side wait ran out in an earlier call; "
+                                     "call moe_check() to clear");
+    if (code)
+        return fail(MOE_ERR_DEVICE_CHECK, "device-side check failed in an earlier call (%d); "
+                                          "call moe_check() to clear", code);
+    return MOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+cudaEvent_t take_event(moe_layer* h) {
+    if (!h->ev_pool.empty()) {
+        cudaEvent_t e = h->ev_pool.back();
+        h->ev_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+// Counts one launch of class `cls` and, with MOE_OPT_KERNEL_TIMING, brackets it
+// with events recorded on the stream the kernel is launched on.
+struct KernelScope {
+    moe_layer* h;
+    int cls;
+    cudaStream_t s;
+    cudaEvent_t a = nullptr;
+    KernelScope(moe_layer* h_, int cls_, cudaStream_t s_) : h(h_), cls(cls_), s(s_) {
+        h->k_launches[cls]++;
+        if (h->timing) {
+            a = take_event(h);
+            if (a) cudaEventRecord(a, s);
+        }
+    }
+    ~KernelScope() {
+        if (!a) return;
+        cudaEvent_t b = take_event(h);
+        if (!b) return;
+        cudaEventRecord(b, s);
+        h->pending.push_back({cls, a, b});
+    }
+};
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_version(void) { return "sparse_moe_b200 0.1 sm_100a"; }
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_OOM: return "out of memory";
+        case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+        case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+        case MOE_ERR_DEVICE_CHECK: return "device-side check failed";
+    }
+    return "unknown status";
+}
+
+const char* moe_last_error(moe_handle) { return g_err; }
+
+moe_status moe_create(const moe_config* cfg, int device, const void* w_router, const void* w_gate,
+                      const void* w_up, const void* w_down, const void* ws_gate,
+                      const void* ws_up, const void* ws_down, const void* rms_weight,
+                      moe_handle* out) {
+    if (!cfg || !out) return fail(MOE_ERR_INVALID_ARG, "cfg and out must not be NULL");
+    *out = nullptr;
+    const moe_config& c = *cfg;
+    if (c.hidden <= 0 || c.n_experts <= 0 || c.n_experts > 1024 || c.top_k <= 0 ||
+        c.top_k > c.n_experts || c.top_k > 16 || c.expert_inter <= 0 || c.shared_inter < 0)
+        return fail(MOE_ERR_INVALID_ARG, "bad layer sizes");
+    if (c.dtype != MOE_DTYPE_F32 && c.dtype != MOE_DTYPE_BF16)
+        return fail(MOE_ERR_INVALID_ARG, "dtype must be MOE_DTYPE_F32 or MOE_DTYPE_BF16");
+    if (c.norm_topk_prob != 1)
+        return fail(MOE_ERR_UNSUPPORTED, "only norm_topk_prob = 1 is implemented");
+    if (!w_router || !w_gate || !w_up || !w_down)
+        return fail(MOE_ERR_INVALID_ARG, "routed weights must not be NULL");
+    if (c.shared_inter > 0 && (!ws_gate || !ws_up || !ws_down))
+        return fail(MOE_ERR_INVALID_ARG, "shared weights must not be NULL when shared_inter > 0");
+    if (rms_weight && !(c.rms_eps >= 0.f))
+        return fail(MOE_ERR_INVALID_ARG, "rms_eps must be >= 0");
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev)
+        return fail(MOE_ERR_INVALID_ARG, "device %d not available", device);
+    DeviceGuard g(device);
+
+    moe_layer* h = new moe_layer();
+    h->cfg = c;
+    h->d = Dims{c.hidden, c.n_experts, c.top_k, c.expert_inter, c.shared_inter};
+    h->device = device;
+    h->dtype = c.dtype == MOE_DTYPE_F32 ? 0 : 1;
+    h->esz = h->dtype == 0 ? 4 : 2;
+    cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, device);
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device);
+    h->tc_ok = h->dtype == 1 && major == 10 && minor == 0 && c.hidden % 128 == 0 &&
+               c.expert_inter % 128 == 0 && c.shared_inter % 128 == 0;
+
+    const size_t H = c.hidden, E = c.n_experts, I = c.expert_inter, Is = c.shared_inter;
+    const size_t es = h->esz;
+    moe_status st = MOE_OK;
+    auto chk = [&](moe_status s) { if (st == MOE_OK) st = s; };
+    chk(copy_weight(&h->w_router, w_router, E * H * es));
+    chk(copy_weight(&h->w_gate, w_gate, E * I * H * es));
+    chk(copy_weight(&h->w_up, w_up, E * I * H * es));
+    chk(copy_weight(&h->w_down, w_down, E * H * I * es));
+    if (Is) {
+        chk(copy_weight(&h->ws_gate, ws_gate, Is * H * es));
+        chk(copy_weight(&h->ws_up, ws_up, Is * H * es));
+        chk(copy_weight(&h->ws_down, ws_down, H * Is * es));
+    }
+    if (rms_weight) chk(copy_weight(&h->rms_w, rms_weight, H * es));
+    if (st == MOE_OK) {
+        cudaError_t e = cudaMalloc(&h->err_dev, sizeof(int));
+        if (e == cudaSuccess) e = cudaMemset(h->err_dev, 0, sizeof(int));
+        if (e == cudaSuccess) e = cudaHostAlloc(&h->err_host, sizeof(int), cudaHostAllocMapped);
+        if (e == cudaSuccess) *h->err_host = 0;
+        if (e == cudaSuccess) e = cudaHostGetDevicePointer(&h->err_host_dev, h->err_host, 0);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->s2, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming);
+        if (e != cudaSuccess)
+            chk(fail(e == cudaErrorMemoryAllocation ? MOE_ERR_OOM : MOE_ERR_CUDA, "create: %s",
+                     cudaGetErrorString(e)));
+    }
+    if (st == MOE_OK && h->tc_ok) {
+        chk(make_map(&h->routed_maps.a_gate, h->w_gate, E * I, H, 128));
+        chk(make_map(&h->routed_maps.a_up, h->w_up, E * I, H, 128));
+        chk(make_map(&h->routed_maps.a_down, h->w_down, E * H, I, 128));
+        if (Is) {
+            chk(make_map(&h->shared_maps.a_gate, h->ws_gate, Is, H, 128));
+            chk(make_map(&h->shared_maps.a_up, h->ws_up, Is, H, 128));
+            chk(make_map(&h->shared_maps.a_down, h->ws_down, H, Is, 128));
+        }
+    }
+    if (st != MOE_OK) {
+        char keep[sizeof g_err];
+        memcpy(keep, g_err, sizeof keep);
+        moe_destroy(h);
+        memcpy(g_err, keep, sizeof keep);
+        return st;
+    }
+    *out = h;
+    return MOE_OK;
+}
+
+moe_status moe_reserve(moe_handle h, int max_tokens) {
+    if (!h || max_tokens < 0) return fail(MOE_ERR_INVALID_ARG, "bad handle or max_tokens");
+    if (max_tokens <= h->max_T) return MOE_OK;
+    DeviceGuard g(h->device);
+    CUDA_TRY(cudaDeviceSynchronize());
+    free_workspace(h);
+    const size_t T = max_tokens, H = h->d.H, E = h->d.E, k = h->d.k, I = h->d.I, Is = h->d.Is;
+    const size_t es = h->esz, S = T * k;
+    const size_t nblocks = (T + kRouteBlock - 1) / kRouteBlock;
+    const int max_units = (int)((S + kNarrow - 1) / kNarrow + E);
+    const int max_shared_units = (int)((T + kNarrow - 1) / kNarrow);
+
+    struct Part { void** ptr; size_t bytes; };
+    std::vector<Part> parts = {
+        {(void**)&h->rb.logits, T * E * 4},
+        {(void**)&h->rb.topk_idx, S * 4},
+        {(void**)&h->rb.topk_w, S * 4},
+        {(void**)&h->rb.block_hist, nblocks * E * 4},
+        {(void**)&h->rb.block_off, nblocks * E * 4},
+        {(void**)&h->rb.counts, E * 4},
+        {(void**)&h->rb.offsets, (E + 1) * 4},
+        {(void**)&h->rb.units, (size_t)max_units * sizeof(Unit)},
+        {(void**)&h->rb.n_units, 4},
+        {(void**)&h->rb.token_slot, S * 4},
+        {(void**)&h->rb.slot_token, S * 4},
+        {(void**)&h->rb.slot_expert, S * 4},
+        {(void**)&h->rb.tickets, (nblocks + 1) * 4},
+        {(void**)&h->sync_routed, (2 + (size_t)max_units) * 4},
+        {(void**)&h->sync_shared, (2 + (size_t)max_shared_units) * 4},
+        {&h->x_norm, h->rms_w ? T * H * es : 0},
+        {&h->xp, S * H * es},
+        {&h->hbuf, S * I * es},
+        {&h->obuf, S * H * es},
+        {&h->hs, T * (Is ? Is : 1) * es},
+        {&h->sbuf, T * H * es},
+        {&h->x_stage, T * H * es},
+        {&h->r_stage, T * H * es},
+        {&h->y_stage, T * H * es},
+    };
+    size_t total = 0;
+    for (auto& p : parts) total += align_up(p.bytes ? p.bytes : 16, 256);
+    char* base = nullptr;
+    CUDA_TRY(cudaMalloc(&base, total));
+    CUDA_TRY(cudaMemset(base, 0, total));
+    size_t off = 0;
+    for (auto& p : parts) {
+        *p.ptr = base + off;
+        off += align_up(p.bytes ? p.bytes : 16, 256);
+    }
+    if (!h->rms_w) h->x_norm = nullptr;
+    h->ws = base;
+    h->max_T = max_tokens;
+    h->max_units = max_units;
+    if (h->tc_ok) {
+        moe_status st = make_map(&h->routed_maps.b_x, h->xp, S, H, 16);
+        if (st == MOE_OK) st = make_map(&h->routed_maps.b_h, h->hbuf, S, I, 16);
+        if (st == MOE_OK && Is) st = make_map(&h->shared_maps.b_h, h->hs, T, Is, 16);
+        if (st != MOE_OK) { free_workspace(h); return st; }
+    }
+    return MOE_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+int choose_width(const moe_layer* h, int T) {
+    return (int64_t)T * h->d.k > (int64_t)16 * h->d.E ? kWide : kNarrow;
+}
+
+moe_status run_shared(moe_layer* h, const void* x_in, int T, cudaStream_t s) {
+    const Dims& d = h->d;
+    if (!d.Is) return MOE_OK;
+    if (h->tc_ok && !h->force_simt) {
+        TcMaps maps = h->shared_maps;
+        moe_status st = make_map(&maps.b_x, x_in, (uint64_t)T, d.H, 16);
+        if (st != MOE_OK) return st;
+        const int width = choose_width(h, T);
+        TcArgs a{};
+        a.H = d.H; a.I = d.Is; a.phases = h->fuse ? 3 : 1;
+        a.dense_T = T; a.unit_width = width;
+        a.units = nullptr; a.n_units = nullptr;
+        a.sync = h->sync_shared; a.hbuf = h->hs; a.out = h->sbuf;
+        a.st = h->status(); a.wait_limit_ns = h->wait_limit_ns; a.inject_stuck = 0;
+        const int units = (T + width - 1) / width;
+        const int tiles = units * (d.Is / 128 + d.H / 128);
+        {
+            KernelScope ks(h, MOE_KERNEL_SHARED, s);
+            CUDA_TRY(launch_tc_experts(maps, a, width, std::min(tiles, h->num_sms), s));
+        }
+        if (!h->fuse) {
+            a.phases = 2;
+            KernelScope ks(h, MOE_KERNEL_SHARED, s);
+            CUDA_TRY(launch_tc_experts(maps, a, width, std::min(tiles, h->num_sms), s));
+        }
+    } else {
+        {
+            KernelScope ks(h, MOE_KERNEL_SHARED, s);
+            CUDA_TRY(launch_simt_gate_up(h->dtype, x_in, h->ws_gate, h->ws_up, nullptr, nullptr,
+                                         T, d.H, d.Is, h->hs, s));
+        }
+        KernelScope ks(h, MOE_KERNEL_SHARED, s);
+        CUDA_TRY(launch_simt_down(h->dtype, h->hs, h->ws_down, nullptr, nullptr, T, d.H, d.Is,
+                                  h->sbuf, s));
+    }
+    return MOE_OK;
+}
+
+moe_status run_layer(moe_layer* h, const void* x, const void* residual, void* y, int T,
+                     int32_t* idx_out, float* w_out, cudaStream_t s) {
+    const Dims& d = h->d;
+    const bool tc = h->tc_ok && !h->force_simt;
+    const int width = choose_width(h, T);
+    RouteBufs rb = h->rb;
+    if (idx_out) rb.topk_idx = idx_out;
+    if (w_out) rb.topk_w = w_out;
+    const void* x_in = h->rms_w ? h->x_norm : x;
+    const bool side = h->shared_stream && d.Is > 0;
+
+    if (side && !h->rms_w) {     // the shared expert needs only x: start it right away
+        CUDA_TRY(cudaEventRecord(h->ev_fork, s));
+        CUDA_TRY(cudaStreamWaitEvent(h->s2, h->ev_fork, 0));
+        moe_status st = run_shared(h, x_in, T, h->s2);
+        if (st != MOE_OK) return st;
+        CUDA_TRY(cudaEventRecord(h->ev_join, h->s2));
+    }
+    {
+        KernelScope ks(h, MOE_KERNEL_ROUTER, s);
+        CUDA_TRY(launch_router(h->dtype, x, h->w_router, h->rms_w, h->cfg.rms_eps, h->x_norm, d,
+                               T, kRouteBlock, rb, 1, width, h->max_units, h->status(), s));
+    }
+    if (side && h->rms_w) {      // with a pre-norm it needs the router's normalised x
+        CUDA_TRY(cudaEventRecord(h->ev_fork, s));
+        CUDA_TRY(cudaStreamWaitEvent(h->s2, h->ev_fork, 0));
+        moe_status st = run_shared(h, x_in, T, h->s2);
+        if (st != MOE_OK) return st;
+        CUDA_TRY(cudaEventRecord(h->ev_join, h->s2));
+    }
+    {
+        KernelScope ks(h, MOE_KERNEL_PERMUTE, s);
+        CUDA_TRY(launch_permute(h->dtype, x_in, h->xp, d, T, kRouteBlock, rb, s));
+    }
+    const int S = T * d.k;
+    if (tc) {
+        TcArgs a{};
+        a.H = d.H; a.I = d.I; a.phases = h->fuse ? 3 : 1;
+        a.dense_T = 0; a.unit_width = width;
+        a.units = rb.units; a.n_units = rb.n_units;
+        a.sync = h->sync_routed; a.hbuf = h->hbuf; a.out = h->obuf;
+        a.st = h->status(); a.wait_limit_ns = h->wait_limit_ns;
+        a.inject_stuck = h->inject_stuck && h->fuse;
+        const int max_units = std::min(h->max_units, (S + width - 1) / width + d.E);
+        const int tiles = max_units * (d.I / 128 + d.H / 128);
+        const int grid = std::min(tiles, h->num_sms);
+        {
+            KernelScope ks(h, MOE_KERNEL_EXPERTS, s);
+            CUDA_TRY(launch_tc_experts(h->routed_maps, a, width, grid, s));
+        }
+        if (!h->fuse) {
+            a.phases = 2;
+            KernelScope ks(h, MOE_KERNEL_EXPERTS, s);
+            CUDA_TRY(launch_tc_experts(h->routed_maps, a, width, grid, s));
+        }
+        h->inject_stuck = 0;
+    } else {
+        const int32_t* n_rows = rb.offsets + d.E;
+        {
+            KernelScope ks(h, MOE_KERNEL_EXPERTS, s);
+            CUDA_TRY(launch_simt_gate_up(h->dtype, h->xp, h->w_gate, h->w_up, rb.slot_expert,
+                                         n_rows, S, d.H, d.I, h->hbuf, s));
+        }
+        KernelScope ks(h, MOE_KERNEL_EXPERTS, s);
+        CUDA_TRY(launch_simt_down(h->dtype, h->hbuf, h->w_down, rb.slot_expert, n_rows, S, d.H,
+                                  d.I, h->obuf, s));
+    }
+    if (d.Is > 0) {
+        if (side) {
+            CUDA_TRY(cudaStreamWaitEvent(s, h->ev_join, 0));
+        } else {
+            moe_status st = run_shared(h, x_in, T, s);
+            if (st != MOE_OK) return st;
+        }
+    }
+    {
+        KernelScope ks(h, MOE_KERNEL_COMBINE, s);
+        CUDA_TRY(launch_combine(h->dtype, h->obuf, d.Is > 0 ? h->sbuf : nullptr, residual, y,
+                                rb.topk_w, rb.token_slot, d, T, s));
+    }
+    h->last_T = T;
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_route(moe_handle h, const void* x, int T, int32_t* topk_idx, float* topk_w,
+                     void* stream) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "NULL handle");
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0");
+    if (T == 0) return MOE_OK;
+    if (!x || !topk_idx || !topk_w) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if (T > h->max_T) return fail(MOE_ERR_INVALID_ARG, "T=%d exceeds reserved %d", T, h->max_T);
+    moe_status pe = pending_device_error(h);
+    if (pe != MOE_OK) return pe;
+    DeviceGuard g(h->device);
+    RouteBufs rb = h->rb;
+    rb.topk_idx = topk_idx;
+    rb.topk_w = topk_w;
+    KernelScope ks(h, MOE_KERNEL_ROUTER, (cudaStream_t)stream);
+    CUDA_TRY(launch_router(h->dtype, x, h->w_router, h->rms_w, h->cfg.rms_eps, nullptr, h->d, T,
+                           kRouteBlock, rb, 0, kNarrow, h->max_units, h->status(),
+                           (cudaStream_t)stream));
+    return MOE_OK;
+}
+
+moe_status moe_forward(moe_handle h, const void* x, const void* residual, void* y, int T,
+                       int32_t* topk_idx_out, float* topk_w_out, void* stream) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "NULL handle");
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0");
+    if (T == 0) return MOE_OK;
+    if (!x || !y) return fail(MOE_ERR_INVALID_ARG, "x and y must not be NULL");
+    if (!aligned16(x) || !aligned16(y) || (residual && !aligned16(residual)))
+        return fail(MOE_ERR_INVALID_ARG, "x, residual and y must be 16-byte aligned");
+    if (T > h->max_T) return fail(MOE_ERR_INVALID_ARG, "T=%d exceeds reserved %d", T, h->max_T);
+    moe_status pe = pending_device_error(h);
+    if (pe != MOE_OK) return pe;
+    DeviceGuard g(h->device);
+    return run_layer(h, x, residual, y, T, topk_idx_out, topk_w_out, (cudaStream_t)stream);
+}
+
+moe_status moe_forward_host(moe_handle h, const void* x_host, const void* residual_host,
+                            void* y_host, int T, void* stream) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "NULL handle");
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0");
+    if (T == 0) return MOE_OK;
+    if (!x_host || !y_host) return fail(MOE_ERR_INVALID_ARG, "x_host and y_host must not be NULL");
+    if (T > h->max_T) return fail(MOE_ERR_INVALID_ARG, "T=%d exceeds reserved %d", T, h->max_T);
+    moe_status pe = pending_device_error(h);
+    if (pe != MOE_OK) return pe;
+    DeviceGuard g(h->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t bytes = (size_t)T * h->d.H * h->esz;
+    CUDA_TRY(cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, s));
+    if (residual_host)
+        CUDA_TRY(cudaMemcpyAsync(h->r_stage, residual_host, bytes, cudaMemcpyHostToDevice, s));
+    moe_status st = run_layer(h, h->x_stage, residual_host ? h->r_stage : nullptr, h->y_stage, T,
+                              nullptr, nullptr, s);
+    if (st != MOE_OK) return st;
+    CUDA_TRY(cudaMemcpyAsync(y_host, h->y_stage, bytes, cudaMemcpyDeviceToHost, s));
+    CUDA_TRY(cudaStreamSynchronize(s));
+    return MOE_OK;
+}
+
+moe_status moe_last_routing(moe_handle h, int32_t* counts, int32_t* offsets, int32_t* token_slot,
+                            void* stream) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "NULL handle");
+    if (!h->ws) return fail(MOE_ERR_INVALID_ARG, "no workspace reserved");
+    DeviceGuard g(h->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    CUDA_TRY(cudaStreamSynchronize(s));
+    if (counts)
+        CUDA_TRY(cudaMemcpy(counts, h->rb.counts, h->d.E * 4, cudaMemcpyDeviceToHost));
+    if (offsets)
+        CUDA_TRY(cudaMemcpy(offsets, h->rb.offsets, (h->d.E + 1) * 4, cudaMemcpyDeviceToHost));
+    if (token_slot && h->last_T)
+        CUDA_TRY(cudaMemcpy(token_slot, h->rb.token_slot, (size_t)h->last_T * h->d.k * 4,
+                            cudaMemcpyDeviceToHost));
+    return MOE_OK;
+}
+
+moe_status moe_check(moe_handle h, void* stream) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "NULL handle");
+    DeviceGuard g(h->device);
+    CUDA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
+    CUDA_TRY(cudaStreamSynchronize(h->s2));
+    int code = 0;
+    CUDA_TRY(cudaMemcpy(&code, h->err_dev, sizeof(int), cudaMemcpyDeviceToHost));
+    if (!code) code = *(volatile int*)h->err_host;
+    CUDA_TRY(cudaMemset(h->err_dev, 0, sizeof(int)));
+    *(volatile int*)h->err_host = 0;
+    if (code == MOE_ERR_TIMEOUT) return fail(MOE_ERR_TIMEOUT, "a bounded device-side wait ran out");
+    if (code) return fail(MOE_ERR_DEVICE_CHECK, "device-side check failed (%d)", code);
+    return MOE_OK;
+}
+
+moe_status moe_set_option(moe_handle h, moe_option opt, int64_t value) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "NULL handle");
+    switch (opt) {
+        case MOE_OPT_WAIT_LIMIT_NS:
+            if (value < 0) return fail(MOE_ERR_INVALID_ARG, "wait limit < 0");
+            h->wait_limit_ns = (uint64_t)value;
+            return MOE_OK;
+        case MOE_OPT_INJECT_STUCK_WAIT: h->inject_stuck = value != 0; return MOE_OK;
+        case MOE_OPT_SHARED_STREAM: h->shared_stream = value != 0; return MOE_OK;
+        case MOE_OPT_FUSE_PHASES: h->fuse = value != 0; return MOE_OK;
+        case MOE_OPT_FORCE_SIMT: h->force_simt = value != 0; return MOE_OK;
+        case MOE_OPT_KERNEL_TIMING: h->timing = value != 0; return MOE_OK;
+    }
+    return fail(MOE_ERR_INVALID_ARG, "unknown option %d", (int)opt);
+}
+
+moe_status moe_kernel_stats(moe_handle h, double* total_ms, int64_t* launches, int reset) {
+    if (!h) return fail(MOE_ERR_INVALID_ARG, "NULL handle");
+    DeviceGuard g(h->device);
+    CUDA_TRY(cudaDeviceSynchronize());
+    for (auto& p : h->pending) {
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) h->k_ms[p.cls] += ms;
+        h->ev_pool.push_back(p.a);
+        h->ev_pool.push_back(p.b);
+    }
+    h->pending.clear();
+    for (int c = 0; c < MOE_KERNEL_CLASSES; ++c) {
+        if (total_ms) total_ms[c] = h->k_ms[c];
+        if (launches) launches[c] = h->k_launches[c];
+        if (reset) { h->k_ms[c] = 0.0; h->k_launches[c] = 0; }
+    }
+    return MOE_OK;
+}
+
+moe_status moe_destroy(moe_handle h) {
+    if (!h) return MOE_OK;
+    DeviceGuard g(h->device);
+    if (h->s2) cudaStreamSynchronize(h->s2);
+    cudaDeviceSynchronize();
+    for (auto& p : h->pending) { cudaEventDestroy(p.a); cudaEventDestroy(p.b); }
+    for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
+    free_workspace(h);
+    void* bufs[] = {h->w_router, h->w_gate, h->w_up, h->w_down, h->ws_gate,
+                    h->ws_up,    h->ws_down, h->rms_w, h->err_dev};
+    for (void* p : bufs)
+        if (p) cudaFree(p);
+    if (h->err_host) cudaFreeHost(h->err_host);
+    if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+    if (h->ev_join) cudaEventDestroy(h->ev_join);
+    if (h->s2) cudaStreamDestroy(h->s2);
+    delete h;
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import json
 import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -32,9 +33,13 @@ SKEW_FILE = os.path.join(GOLDEN_DIR, "skew_talker_prefill_skewed.json")
 
 def bf16_bits(a: np.ndarray) -> np.ndarray:
     """Round float32 (or float64 via float32) values to bf16, nearest-even; returns uint16 bits."""
-    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
-    lsb = (u >> np.uint32(16)) & np.uint32(1)
-    return ((u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)).astype(np.uint16)
+    u = np.array(a, dtype=np.float32, copy=True).view(np.uint32)
+    lsb = u >> np.uint32(16)
+    lsb &= np.uint32(1)
+    u += lsb
+    u += np.uint32(0x7FFF)
+    u >>= np.uint32(16)
+    return u.astype(np.uint16)
 
 
 def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
@@ -184,8 +189,9 @@ def make(name: str, T: int | None = None) -> Inputs:
         return make_skewed(wl, T, p["s"], p["dead_steps"], p.get("hot_bias", 0.05))
     if wl.n_layers > 1:
         x = _store(wl, _normal(np.random.default_rng((wl.seed, 0)), (T, wl.H), wl.x_scale))
-        layers = [draw_layer_weights(wl, np.random.default_rng((wl.seed, 1 + l)))
-                  for l in range(wl.n_layers)]
+        with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+            layers = list(ex.map(lambda l: draw_layer_weights(
+                wl, np.random.default_rng((wl.seed, 1 + l))), range(wl.n_layers)))
         return Inputs(wl, x, layers)
     rng = np.random.default_rng(wl.seed)
     x = _store(wl, _normal(rng, (T, wl.H), wl.x_scale))

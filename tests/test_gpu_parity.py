@@ -1,0 +1,251 @@
+"""CUDA path vs the fp64 oracle, through the C ABI, on the same seeded inputs."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests.parity import assert_parity, compare
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+smt = pytest.importorskip("sparse_moe_transformer_b200")
+
+
+def _cfg(wl, k=None):
+    return smt.LayerConfig(wl.H, wl.E, k or wl.k, wl.I, wl.Is, wl.dtype, wl.rms_eps)
+
+
+def _layer(inp, li=0, **opts):
+    wl = inp.workload
+    L = inp.layers[li]
+    layer = smt.MoELayer.from_numpy(_cfg(wl), L.arrays(), device=0)
+    for k, v in opts.items():
+        layer.set_option(k, v)
+    orc = oracle.Oracle(oracle.LayerWeights(**L.arrays(), top_k=wl.k, rms_eps=wl.rms_eps))
+    return layer, orc
+
+
+def _values(t):
+    a = smt.to_numpy(t)
+    return synth.bf16_to_f32(a) if a.dtype == np.uint16 else a
+
+
+def _run(layer, x_np, residual=None, **kw):
+    x = smt.to_device(x_np)
+    r = None if residual is None else smt.to_device(residual)
+    y, idx, w = layer.forward(x, residual=r, return_routing=True, **kw)
+    torch.cuda.synchronize()
+    assert layer.check() == 0
+    return _values(y), idx.cpu().numpy(), w.cpu().numpy()
+
+
+def test_tiny_fp32():
+    inp = synth.make("tiny_fp32")
+    layer, orc = _layer(inp)
+    y, idx, w = _run(layer, inp.x)
+    rep = compare(orc, inp.x, y, idx, w, "f32")
+    assert_parity(rep, "f32")
+    assert rep.near_ties == 0 and np.array_equal(idx, orc.forward(inp.x)[1])
+
+
+def test_decode_bf16():
+    inp = synth.make("talker_decode")
+    layer, orc = _layer(inp)
+    y, idx, w = _run(layer, inp.x)
+    rep = compare(orc, inp.x, y, idx, w, "bf16")
+    assert_parity(rep, "bf16")
+
+
+SHAPES = [  # H, E, k, I, Is, T   (narrow and wide tile paths, ragged tails, k=1, no shared)
+    (256, 16, 4, 128, 128, 37),
+    (256, 8, 2, 256, 256, 1200),
+    (128, 4, 1, 128, 0, 5),
+    (256, 16, 4, 128, 128, 1),
+    (384, 32, 8, 256, 384, 200),
+    (256, 64, 6, 128, 256, 333),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "H{}_E{}_k{}_I{}_Is{}_T{}".format(*s))
+def test_bf16_shapes(shape):
+    H, E, k, I, Is, T = shape
+    inp = synth.make_custom(H, E, k, I, Is, T, "bf16", seed=5)
+    layer, orc = _layer(inp)
+    y, idx, w = _run(layer, inp.x)
+    assert_parity(compare(orc, inp.x, y, idx, w, "bf16"), "bf16")
+
+
+@pytest.mark.parametrize("shape", [(8, 6, 2, 16, 32, 50), (64, 8, 3, 32, 48, 77)])
+def test_fp32_shapes(shape):
+    H, E, k, I, Is, T = shape
+    inp = synth.make_custom(H, E, k, I, Is, T, "f32", seed=6, w_scale=0.3)
+    layer, orc = _layer(inp)
+    y, idx, w = _run(layer, inp.x)
+    assert_parity(compare(orc, inp.x, y, idx, w, "f32"), "f32")
+
+
+def _sampled(name, n=64, seed=0):
+    inp = synth.make(name)
+    layer, orc = _layer(inp)
+    y, idx, w = _run(layer, inp.x)
+    T = inp.x.shape[0]
+    rows = np.sort(np.random.default_rng(seed).choice(T, n, replace=False))
+    rows = np.unique(np.concatenate([rows, [0, T - 1]]))
+    rep = compare(orc, inp.x, y[rows], idx[rows], w[rows], "bf16", rows=rows)
+    assert_parity(rep, "bf16")
+    return inp, layer, idx
+
+
+def test_prefill_sampled():
+    inp, layer, idx = _sampled("talker_prefill")
+    counts, offsets, slots = layer.last_routing(inp.x.shape[0])
+    assert np.array_equal(counts, np.bincount(idx.ravel(), minlength=inp.workload.E))
+
+
+def test_skewed_sampled():
+    inp, layer, idx = _sampled("talker_prefill_skewed")
+    counts = np.bincount(idx.ravel(), minlength=inp.workload.E)
+    assert (counts == 0).sum() >= 40
+    share = counts[inp.skew["hot"]].sum() / idx.size
+    assert abs(share - 0.70) < 0.02
+    assert counts[inp.skew["dead"]].sum() == 0
+
+
+def test_stack20(record_property):
+    """20 pre-RMSNorm MoE layers with residual adds, T=64.
+
+    Reference: the fp64 oracle layer by layer, with the hidden state stored in
+    bf16 between layers (the Talker's activations are bf16 tensors; each layer is
+    exact on its stored input).  Checked two ways: (1) teacher-forced, every
+    layer's oracle on the GPU's own bf16 input to that layer; (2) end to end, the
+    oracle stack from the same first input.  The drift of the GPU stack from a
+    stack that never rounds the hidden state is recorded, not asserted: bf16
+    rounding of the residual stream plus routing flips at near ties put it
+    around 3e-2 after 20 layers."""
+    inp = synth.make("talker_stack20")
+    wl = inp.workload
+    h_gpu = smt.to_device(inp.x)
+    h_ref = inp.x.copy()                                          # bf16 bits
+    h_f64 = synth.bf16_to_f32(inp.x).astype(np.float64)
+    worst = 0.0
+    for L in inp.layers:
+        layer = smt.MoELayer.from_numpy(_cfg(wl), L.arrays(), device=0)
+        orc = oracle.Oracle(oracle.LayerWeights(**L.arrays(), top_k=wl.k, rms_eps=wl.rms_eps))
+        x_in = smt.to_numpy(h_gpu)
+        y, idx, w = layer.forward(h_gpu, residual=h_gpu, return_routing=True)
+        torch.cuda.synchronize()
+        assert layer.check() == 0
+        rep = compare(orc, x_in, _values(y), idx.cpu().numpy(), w.cpu().numpy(), "bf16",
+                      residual=x_in)
+        assert_parity(rep, "bf16")
+        worst = max(worst, rep.rel_err)
+        y_ref, _, _, _ = orc.forward(h_ref, residual=h_ref)
+        h_ref = synth.bf16_bits(y_ref)
+        h_f64 = h_f64 + _oracle_f64(L, wl).forward(h_f64)[0]
+        h_gpu = y
+        layer.close()
+    out = _values(h_gpu)
+    ref = synth.bf16_to_f32(h_ref).astype(np.float64)
+    err = np.max(np.abs(out - ref)) / np.max(np.abs(ref))
+    drift = np.max(np.abs(out - h_f64)) / np.max(np.abs(h_f64))
+    record_property("stack_rel_err", float(err))
+    record_property("worst_layer_rel_err", float(worst))
+    record_property("fp64_stream_drift", float(drift))
+    assert err <= 2e-2, (err, worst, drift)
+
+
+def _oracle_f64(L, wl):
+    """Oracle of one layer with its weights widened exactly to fp64 (for fp64 inputs)."""
+    f64 = {k: (synth.bf16_to_f32(v).astype(np.float64) if v.dtype == np.uint16 else v)
+           for k, v in L.arrays().items()}
+    return oracle.Oracle(oracle.LayerWeights(**f64, top_k=wl.k, rms_eps=wl.rms_eps))
+
+
+def test_route_only_matches_forward():
+    inp = synth.make("talker_decode")
+    layer, orc = _layer(inp)
+    x = smt.to_device(inp.x)
+    idx, w = layer.route(x)
+    _, idx2, w2 = layer.forward(x, return_routing=True)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2) and torch.equal(w, w2)
+    _, idx_ref, w_ref, gap = orc.route(inp.x)
+    ok = gap > 1e-3
+    assert np.array_equal(idx.cpu().numpy()[ok], idx_ref[ok])
+    assert np.max(np.abs(w.cpu().numpy()[ok] - w_ref[ok])) <= 2e-5
+    assert np.all(np.abs(w.cpu().numpy().sum(1) - 1) < 1e-6)
+
+
+def test_paths_agree():
+    inp = synth.make_custom(256, 16, 4, 256, 128, 300, "bf16", seed=9)
+    outs = {}
+    for name, opts in {"fused": {}, "unfused": {"fuse_phases": 0},
+                       "one_stream": {"shared_stream": 0}, "simt": {"force_simt": 1}}.items():
+        layer, orc = _layer(inp, **opts)
+        y, idx, w = _run(layer, inp.x)
+        assert_parity(compare(orc, inp.x, y, idx, w, "bf16"), "bf16")
+        outs[name] = y
+    assert np.array_equal(outs["fused"], outs["unfused"])
+    assert np.array_equal(outs["fused"], outs["one_stream"])
+
+
+def test_residual_in_place_and_host_path():
+    inp = synth.make("talker_decode")
+    layer, orc = _layer(inp)
+    r_np = synth.make_tokens(inp.workload, 8, seed=1)
+    x = smt.to_device(inp.x)
+    r = smt.to_device(r_np)
+    y_ref, idx, w = layer.forward(x, residual=r, return_routing=True)
+    assert_parity(compare(orc, inp.x, _values(y_ref), idx.cpu().numpy(), w.cpu().numpy(), "bf16",
+                          residual=r_np), "bf16")
+    layer.forward(x, residual=r, out=r)          # y aliases the residual
+    torch.cuda.synchronize()
+    assert torch.equal(r, y_ref)
+    xh = torch.from_numpy(inp.x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    layer.forward_host(xh, yh)
+    y_dev = layer.forward(x)
+    torch.cuda.synchronize()
+    assert torch.equal(yh, y_dev.cpu())
+
+
+def test_permutation_bookkeeping():
+    inp = synth.make_custom(256, 16, 4, 128, 128, 257, "bf16", seed=11)
+    layer, orc = _layer(inp)
+    y, idx, w = _run(layer, inp.x)
+    T, k, E = 257, 4, 16
+    counts, offsets, slots = layer.last_routing(T)
+    assert np.array_equal(counts, np.bincount(idx.ravel(), minlength=E))
+    assert np.array_equal(offsets, np.concatenate([[0], np.cumsum(counts)]))
+    assert np.array_equal(np.sort(slots.ravel()), np.arange(T * k))   # a bijection
+    for e in range(E):                        # rows of one expert in token order
+        toks = [t for t in range(T) for j in range(k) if idx[t, j] == e]
+        rows = [slots[t, j] for t in range(T) for j in range(k) if idx[t, j] == e]
+        assert rows == list(range(offsets[e], offsets[e + 1]))
+        assert toks == sorted(toks)
+
+
+def test_zero_tokens_and_growth():
+    inp = synth.make_custom(256, 16, 4, 128, 128, 40, "bf16", seed=12)
+    layer, orc = _layer(inp)
+    x = smt.to_device(inp.x)
+    y = torch.empty_like(x)
+    assert layer.lib.moe_forward(layer.handle, x.data_ptr(), None, y.data_ptr(), 0, None, None,
+                                 None) == 0
+    layer.reserve(8)
+    ys, idx, w = _run(layer, inp.x)          # grows the workspace to 40 tokens
+    assert_parity(compare(orc, inp.x, ys, idx, w, "bf16"), "bf16")
+
+
+def test_bounded_wait_reports_timeout_and_recovers():
+    inp = synth.make_custom(256, 16, 4, 128, 128, 64, "bf16", seed=13)
+    layer, orc = _layer(inp)
+    layer.set_option("wait_limit_ns", 2_000_000)      # 2 ms
+    layer.set_option("inject_stuck_wait", 1)          # a dependency count that is never reached
+    x = smt.to_device(inp.x)
+    layer.forward(x)
+    assert layer.check() == smt.MOE_ERR_TIMEOUT
+    layer.set_option("wait_limit_ns", 1_000_000_000)
+    y, idx, w = _run(layer, inp.x)                    # the context is still usable
+    assert_parity(compare(orc, inp.x, y, idx, w, "bf16"), "bf16")
