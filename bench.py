@@ -352,7 +352,8 @@ def main():
         # every launch the library made while capturing is a kernel node of the graph
         launches_per_step = sum(n for hs in handles for layer in hs
                                 for n, _ in layer.kernel_stats(reset=True).values()) / cycle
-        graph.replay()
+        with torch.cuda.stream(stream):
+            graph.replay()
         torch.cuda.synchronize()
     n_rep = max(1, -(-K // cycle)) if use_graph else K
     steps_timed = n_rep * cycle if use_graph else K
@@ -369,8 +370,9 @@ def main():
     with ClockSampler(gpu_uuid) as clocks:
         start.record(stream)
         if use_graph:
-            for _ in range(n_rep):
-                graph.replay()
+            with torch.cuda.stream(stream):      # replay on the stream the events time
+                for _ in range(n_rep):
+                    graph.replay()
         else:
             with torch.cuda.stream(stream):
                 for i in range(K):
@@ -399,9 +401,9 @@ def main():
             layer.set_option("kernel_timing", 1)
     done = 0
     while done < kt_steps:
-        burst = min(32, kt_steps - done)
+        burst = min(8, kt_steps - done)
         with torch.cuda.stream(stream):
-            torch.cuda._sleep(2_000_000)
+            torch.cuda._sleep(20_000_000)        # ~10 ms: covers the burst's host enqueue
             for i in range(burst):
                 step((done + i) % rotate)
         done += burst

@@ -13,6 +13,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "device.cuh"
 #include "layer.h"
 
@@ -36,17 +38,29 @@ combine_kernel(const T* __restrict__ o, const T* __restrict__ sh, const T* __res
         float acc[VEC];
 #pragma unroll
         for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
-        for (int i = 0; i < k; ++i) {
-            const T* src = o + (size_t)slot[i] * H + j0;
-            T vals[VEC];
-            if (VEC * sizeof(T) == 16) {
-                *reinterpret_cast<uint4*>(vals) = __ldg(reinterpret_cast<const uint4*>(src));
-            } else {
+        // slot rows in groups of 8 with all loads of a group in flight, summed in slot order
+#pragma unroll 1
+        for (int i0 = 0; i0 < k; i0 += 8) {
+            T vals[8][VEC];
 #pragma unroll
-                for (int v = 0; v < VEC; ++v) vals[v] = src[v];
+            for (int i = 0; i < 8; ++i) {
+                if (i0 + i < k) {
+                    const T* src = o + (size_t)slot[i0 + i] * H + j0;
+                    if (VEC * sizeof(T) == 16) {
+                        *reinterpret_cast<uint4*>(vals[i]) = __ldg(reinterpret_cast<const uint4*>(src));
+                    } else {
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) vals[i][v] = src[v];
+                    }
+                }
             }
 #pragma unroll
-            for (int v = 0; v < VEC; ++v) acc[v] = fmaf(wt[i], to_f32(vals[v]), acc[v]);
+            for (int i = 0; i < 8; ++i) {
+                if (i0 + i < k) {
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) acc[v] = fmaf(wt[i0 + i], to_f32(vals[i][v]), acc[v]);
+                }
+            }
         }
         const size_t base = (size_t)t * H + j0;
         if (sh) {
@@ -70,7 +84,7 @@ combine_kernel(const T* __restrict__ o, const T* __restrict__ sh, const T* __res
 }
 
 // h[r][f] = SiLU(x_r . Wg[e][f]) * (x_r . Wu[e][f]), one thread per (row, f).
-template <typename T>
+template <typename T, bool PACKED>
 __global__ void __launch_bounds__(256)
 simt_gate_up_kernel(const T* __restrict__ xin, const T* __restrict__ wg, const T* __restrict__ wu,
                     const int32_t* __restrict__ slot_expert, const int32_t* __restrict__ n_rows,
@@ -81,20 +95,23 @@ simt_gate_up_kernel(const T* __restrict__ xin, const T* __restrict__ wg, const T
         const int r = (int)(idx / I), f = (int)(idx % I);
         const int e = slot_expert ? slot_expert[r] : 0;
         const T* xr = xin + (size_t)r * H;
-        const T* g = wg + ((size_t)e * I + f) * H;
-        const T* u = wu + ((size_t)e * I + f) * H;
         float ag = 0.f, au = 0.f;
         for (int j = 0; j < H; ++j) {
-            float xv = to_f32(xr[j]);
-            ag = fmaf(xv, to_f32(g[j]), ag);
-            au = fmaf(xv, to_f32(u[j]), au);
+            const float xv = to_f32(xr[j]);
+            if (PACKED) {
+                ag = fmaf(xv, to_f32(wg[packed_gu_offset(e, f, j, 0, I, H)]), ag);
+                au = fmaf(xv, to_f32(wg[packed_gu_offset(e, f, j, 1, I, H)]), au);
+            } else {
+                ag = fmaf(xv, to_f32(wg[((size_t)e * I + f) * H + j]), ag);
+                au = fmaf(xv, to_f32(wu[((size_t)e * I + f) * H + j]), au);
+            }
         }
         h[(size_t)r * I + f] = from_f32<T>(silu_exact(ag) * au);
     }
 }
 
 // out[r][j] = h_r . Wd[e][j], one thread per (row, j).
-template <typename T>
+template <typename T, bool PACKED>
 __global__ void __launch_bounds__(256)
 simt_down_kernel(const T* __restrict__ h, const T* __restrict__ wd,
                  const int32_t* __restrict__ slot_expert, const int32_t* __restrict__ n_rows,
@@ -105,10 +122,42 @@ simt_down_kernel(const T* __restrict__ h, const T* __restrict__ wd,
         const int r = (int)(idx / H), j = (int)(idx % H);
         const int e = slot_expert ? slot_expert[r] : 0;
         const T* hr = h + (size_t)r * I;
-        const T* w = wd + ((size_t)e * H + j) * I;
         float a = 0.f;
-        for (int f = 0; f < I; ++f) a = fmaf(to_f32(hr[f]), to_f32(w[f]), a);
+        for (int f = 0; f < I; ++f) {
+            const size_t off = PACKED ? packed_down_offset(e, j, f, H, I) : ((size_t)e * H + j) * I + f;
+            a = fmaf(to_f32(hr[f]), to_f32(wd[off]), a);
+        }
         out[(size_t)r * H + j] = from_f32<T>(a);
+    }
+}
+
+// dst[v] for v over 16-byte vectors of the tile-contiguous layout (see layer.h):
+// vector v holds physical chunk (v & 7) of row r, i.e. logical chunk (v & 7) ^ (r & 7).
+// Gate/up (src1 != nullptr): pair index (e, mt, kb), member = gate / up.
+// Down (src1 == nullptr): pair index (e, mt2, kb), member = row block 2 mt2 + member.
+__global__ void __launch_bounds__(256)
+pack_tiles_kernel(const uint4* __restrict__ src0, const uint4* __restrict__ src1,
+                  uint4* __restrict__ dst, int E, int R, int C, size_t total) {
+    const int MT = R / 128, KB = C / 64;
+    const int NB = src1 ? MT : (MT + 1) / 2;      // row blocks (or block pairs) per expert
+    for (size_t v = blockIdx.x * (size_t)blockDim.x + threadIdx.x; v < total;
+         v += (size_t)gridDim.x * blockDim.x) {
+        const int r = (int)((v >> 3) & 127);
+        const int c8 = (int)(v & 7) ^ (r & 7);
+        size_t rest = v >> 10;
+        const int member = (int)(rest & 1); rest >>= 1;
+        const int kb = (int)(rest % KB); rest /= KB;
+        const int nb = (int)(rest % NB);
+        const int e = (int)(rest / NB);
+        const uint4* src = src0;
+        int mt = nb;
+        if (src1) {
+            src = member ? src1 : src0;
+        } else {
+            mt = 2 * nb + member;
+            if (mt >= MT) continue;                    // the zero-filled odd half
+        }
+        dst[v] = src[(((size_t)e * R + mt * 128 + r) * C + kb * 64) / 8 + c8];
     }
 }
 
@@ -146,34 +195,55 @@ cudaError_t launch_combine(int dtype, const void* o, const void* sh, const void*
 }
 
 cudaError_t launch_simt_gate_up(int dtype, const void* xin, const void* w_gate, const void* w_up,
-                                const int32_t* slot_expert, const int32_t* n_rows_dev,
+                                int packed, const int32_t* slot_expert, const int32_t* n_rows_dev,
                                 int max_rows, int H, int I, void* hbuf, cudaStream_t s) {
     if (max_rows <= 0) return cudaSuccess;
     int grid = simt_grid((size_t)max_rows * I);
+    using bf = __nv_bfloat16;
     if (dtype == 0)
-        simt_gate_up_kernel<float><<<grid, 256, 0, s>>>((const float*)xin, (const float*)w_gate,
-                                                       (const float*)w_up, slot_expert,
-                                                       n_rows_dev, max_rows, H, I, (float*)hbuf);
+        simt_gate_up_kernel<float, false><<<grid, 256, 0, s>>>(
+            (const float*)xin, (const float*)w_gate, (const float*)w_up, slot_expert, n_rows_dev,
+            max_rows, H, I, (float*)hbuf);
+    else if (packed)
+        simt_gate_up_kernel<bf, true><<<grid, 256, 0, s>>>(
+            (const bf*)xin, (const bf*)w_gate, (const bf*)w_up, slot_expert, n_rows_dev, max_rows,
+            H, I, (bf*)hbuf);
     else
-        simt_gate_up_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            (const __nv_bfloat16*)xin, (const __nv_bfloat16*)w_gate, (const __nv_bfloat16*)w_up,
-            slot_expert, n_rows_dev, max_rows, H, I, (__nv_bfloat16*)hbuf);
+        simt_gate_up_kernel<bf, false><<<grid, 256, 0, s>>>(
+            (const bf*)xin, (const bf*)w_gate, (const bf*)w_up, slot_expert, n_rows_dev, max_rows,
+            H, I, (bf*)hbuf);
     return cudaGetLastError();
 }
 
-cudaError_t launch_simt_down(int dtype, const void* hbuf, const void* w_down,
+cudaError_t launch_simt_down(int dtype, const void* hbuf, const void* w_down, int packed,
                              const int32_t* slot_expert, const int32_t* n_rows_dev, int max_rows,
                              int H, int I, void* out, cudaStream_t s) {
     if (max_rows <= 0) return cudaSuccess;
     int grid = simt_grid((size_t)max_rows * H);
+    using bf = __nv_bfloat16;
     if (dtype == 0)
-        simt_down_kernel<float><<<grid, 256, 0, s>>>((const float*)hbuf, (const float*)w_down,
-                                                    slot_expert, n_rows_dev, max_rows, H, I,
-                                                    (float*)out);
+        simt_down_kernel<float, false><<<grid, 256, 0, s>>>(
+            (const float*)hbuf, (const float*)w_down, slot_expert, n_rows_dev, max_rows, H, I,
+            (float*)out);
+    else if (packed)
+        simt_down_kernel<bf, true><<<grid, 256, 0, s>>>((const bf*)hbuf, (const bf*)w_down,
+                                                        slot_expert, n_rows_dev, max_rows, H, I,
+                                                        (bf*)out);
     else
-        simt_down_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            (const __nv_bfloat16*)hbuf, (const __nv_bfloat16*)w_down, slot_expert, n_rows_dev,
-            max_rows, H, I, (__nv_bfloat16*)out);
+        simt_down_kernel<bf, false><<<grid, 256, 0, s>>>((const bf*)hbuf, (const bf*)w_down,
+                                                         slot_expert, n_rows_dev, max_rows, H, I,
+                                                         (bf*)out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_tiles(const void* src0, const void* src1, void* dst, int E, int R, int C,
+                              cudaStream_t s) {
+    if (R % 128 || C % 64) return cudaErrorInvalidValue;
+    const int NB = src1 ? R / 128 : (R / 128 + 1) / 2;
+    const size_t total = (size_t)E * NB * (C / 64) * 2 * 1024;     // 16-byte vectors
+    const int grid = (int)std::min<size_t>((total + 255) / 256, 148 * 32);
+    pack_tiles_kernel<<<grid, 256, 0, s>>>((const uint4*)src0, (const uint4*)src1, (uint4*)dst,
+                                           E, R, C, total);
     return cudaGetLastError();
 }
 

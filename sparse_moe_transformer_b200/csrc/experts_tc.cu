@@ -9,16 +9,22 @@
 // ragged token count costs at most 15 padded columns instead of a 128-row tile.
 //   gate/up tile: D_gate = Wg[e][128 rows] . X^T and D_up = Wu[e][128 rows] . X^T
 //                 share the B operand; the epilogue forms SiLU(D_gate) * D_up.
-//   down tile:    D = Wd[e][128 rows] . Hrows^T.
-// A and B are staged by TMA (128-byte swizzle, no multicast) into a ring of
-// shared-memory stages; one thread issues tcgen05.mma into TMEM accumulators;
-// four epilogue warps read TMEM with tcgen05.ld and store bf16 rows.
+//   down tile:    D_0, D_1 = Wd[e][two 128-row blocks] . Hrows^T (256 outputs),
+//                 the same two-panel shape, so both phases move 32 KB of weights
+//                 per k-step.
+// Weights are pre-packed as the exact 128-byte-swizzled tile images the MMA
+// reads, so each k-step's weights arrive by one contiguous bulk copy; token rows
+// come by TMA (128-byte swizzle, no multicast).  Stages form a shared-memory
+// ring; one thread issues tcgen05.mma into TMEM accumulators; eight epilogue
+// warps read TMEM with tcgen05.ld and store bf16 rows with 16-byte stores.
 //
 // The kernel is persistent: CTAs take tiles from a global counter, gate/up tiles
 // first, then down tiles.  When both phases run in one launch, a down tile of a
 // unit waits (bounded by a time limit) until the unit's gate/up tiles have
 // published their h rows; every gate/up tile is taken before any down tile and
-// never waits, so the wait always ends.  Every wait in the kernel is bounded; a
+// never waits, so the wait always ends.  (Ordering tiles in waves of units --
+// each wave's gate/up then down tiles -- was measured slower: down tiles then
+// hold SMs idle while their wave's gate/up tiles still stream.)  Every wait in the kernel is bounded; a
 // wait that runs out records MOE_ERR_TIMEOUT and the CTA drains and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -32,11 +38,13 @@ namespace {
 
 constexpr int kBM = 128;           // weight rows per tile (MMA M)
 constexpr int kBK = 64;            // K elements per stage: one 128-byte swizzle atom
-constexpr int kThreads = 192;      // warp 0 TMA producer, warp 1 MMA, warps 2-5 epilogue
+constexpr int kEpiWarps = 8;       // two warps per TMEM lane quarter, alternating columns
+constexpr int kThreads = 64 + 32 * kEpiWarps;   // warp 0 producer, warp 1 MMA, epilogue
 constexpr int kRing = 4;           // tile-info ring depth
-constexpr int kABytes = kBM * kBK * 2;
+constexpr int kABytes = kBM * kBK * 2;          // one packed weight tile
 constexpr int kBoxRows = 16;       // activation rows per TMA box
 constexpr int kBoxBytes = kBoxRows * kBK * 2;
+constexpr int kEpiStage = 16 * 32 * 2;          // per-warp transpose buffer: 16 rows x 32 cols
 constexpr uint64_t kDrainLimitNs = 200ull * 1000 * 1000;
 
 constexpr int pow2_at_least(int v) {
@@ -53,9 +61,11 @@ struct TcCfg {
     static constexpr int kBBytes = BN * kBK * 2;
     static constexpr int kStageBytes = 2 * kABytes + kBBytes;
     static constexpr int kCtrlBytes = 1024;
-    static constexpr int kSmem = kStages * kStageBytes + kCtrlBytes + 1024;   // + align slack
+    static constexpr int kSmem =
+        kStages * kStageBytes + kEpiWarps * kEpiStage + kCtrlBytes + 1024;   // + align slack
     static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
     static_assert(kTmemCols <= 512, "TMEM has 512 columns");
+    static_assert(kSmem <= 232448, "shared memory per CTA");
 };
 
 struct Tile {
@@ -70,16 +80,27 @@ struct Tile {
 __device__ __forceinline__ Tile decode_tile(int i, int n_units, const TcArgs& a, int mt_gu,
                                             int mt_dn, int bn) {
     Tile t;
-    const int n_gu = (a.phases & 1) ? n_units * mt_gu : 0;
-    const int n_dn = (a.phases & 2) ? n_units * mt_dn : 0;
-    if (i < n_gu) {
-        t.phase = 0; t.unit = i / mt_gu; t.mt = i - t.unit * mt_gu;
-    } else if (i - n_gu < n_dn) {
-        const int j = i - n_gu;
-        t.phase = 1; t.unit = j / mt_dn; t.mt = j - t.unit * mt_dn;
-    } else {
-        t.phase = -1; t.unit = t.mt = t.expert = t.row_start = t.n_len = 0;
+    if (a.phases == 4) {          // router logits: one two-panel tile (256 experts) per unit
+        if (i < n_units * mt_dn) {
+            t.phase = 2; t.unit = i / mt_dn; t.mt = i - t.unit * mt_dn;
+            t.expert = 0; t.row_start = t.unit * bn; t.n_len = min(bn, a.dense_T - t.row_start);
+        } else {
+            t.phase = -1; t.unit = t.mt = t.expert = t.row_start = t.n_len = 0;
+        }
         return t;
+    }
+    {
+        const int n_gu = (a.phases & 1) ? n_units * mt_gu : 0;
+        const int n_dn = (a.phases & 2) ? n_units * mt_dn : 0;
+        if (i < n_gu) {
+            t.phase = 0; t.unit = i / mt_gu; t.mt = i - t.unit * mt_gu;
+        } else if (i - n_gu < n_dn) {
+            const int j = i - n_gu;
+            t.phase = 1; t.unit = j / mt_dn; t.mt = j - t.unit * mt_dn;
+        } else {
+            t.phase = -1; t.unit = t.mt = t.expert = t.row_start = t.n_len = 0;
+            return t;
+        }
     }
     if (a.dense_T > 0) {
         t.expert = 0;
@@ -92,44 +113,67 @@ __device__ __forceinline__ Tile decode_tile(int i, int n_units, const TcArgs& a,
     return t;
 }
 
+// Wait (bounded) until `flag` reaches `target`; false after recording a timeout.
+__device__ __forceinline__ bool wait_count(const int* flag, int target, const TcArgs& a) {
+    if (ld_acquire_gpu(flag) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_gpu(flag) < target) {
+        __nanosleep(64);
+        if (globaltimer_ns() - t0 > a.wait_limit_ns) {
+            report_error(a.st, kErrTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
 template <int BN>
 __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs& a) {
     using C = TcCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint8_t* ctrl = smem + C::kStages * C::kStageBytes;
+    uint8_t* epi_smem = smem + C::kStages * C::kStageBytes;
+    uint8_t* ctrl = epi_smem + kEpiWarps * kEpiStage;
     uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
     uint64_t* empty = full + C::kStages;
     uint64_t* accfull = empty + C::kStages;
     uint64_t* accempty = accfull + C::kAcc;
     uint64_t* tfull = accempty + C::kAcc;
     uint64_t* tempty = tfull + kRing;
-    uint64_t* pubbar = tempty + kRing;      // 4 epilogue warps finished a gate/up tile
+    uint64_t* pubbar = tempty + kRing;      // epilogue warps finished a gate/up tile
     uint64_t* drainbar = pubbar + 1;        // all MMAs of this CTA completed
     Tile* ring = reinterpret_cast<Tile*>(drainbar + 1);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring + kRing);
     int* s_misc = reinterpret_cast<int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int mt_gu = a.I / kBM, mt_dn = a.H / kBM;
+    const bool router = a.phases == 4;
+    const int mt_gu = a.I / kBM;                      // gate/up tiles: 128 features each
+    // down tiles: 256 output features each; router tiles: 256 experts each
+    const int mt_dn = router ? (a.I / kBM + 1) / 2 : (a.H / kBM + 1) / 2;
+    const int kb_gu = a.H / kBK, kb_dn = router ? a.H / kBK : a.I / kBK;
     int* tile_counter = a.sync;
     int* exit_counter = a.sync + 1;
     int* done = a.sync + 2;
     const uint64_t limit = a.wait_limit_ns;
+    const bool fused = (a.phases & 3) == 3;
 
     const int n_units = a.dense_T > 0 ? (a.dense_T + BN - 1) / BN : *a.n_units;
-    const int n_tiles = n_units * (((a.phases & 1) ? mt_gu : 0) + ((a.phases & 2) ? mt_dn : 0));
+    const int n_tiles = router ? n_units * mt_dn
+                               : n_units * (((a.phases & 1) ? mt_gu : 0) + ((a.phases & 2) ? mt_dn : 0));
 
     if (tid == 0) {
-        for (int s = 0; s < C::kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        for (int s = 0; s < C::kAcc; ++s) { mbar_init(&accfull[s], 1); mbar_init(&accempty[s], 4); }
-        for (int s = 0; s < kRing; ++s) { mbar_init(&tfull[s], 1); mbar_init(&tempty[s], 5); }
-        mbar_init(pubbar, 4);
+        for (int s = 0; s < C::kStages; ++s) { mbar_init(&full[s], 2); mbar_init(&empty[s], 1); }
+        for (int s = 0; s < C::kAcc; ++s) {
+            mbar_init(&accfull[s], 1);
+            mbar_init(&accempty[s], kEpiWarps);
+        }
+        for (int s = 0; s < kRing; ++s) { mbar_init(&tfull[s], 1); mbar_init(&tempty[s], 1 + kEpiWarps); }
+        mbar_init(pubbar, kEpiWarps);
         mbar_init(drainbar, 1);
         mbar_fence_init();
-        tma_prefetch_desc(&maps.a_gate); tma_prefetch_desc(&maps.a_up);
-        tma_prefetch_desc(&maps.a_down); tma_prefetch_desc(&maps.b_x);
+        tma_prefetch_desc(&maps.b_x);
         tma_prefetch_desc(&maps.b_h);
     }
     if (warp == 1) tmem_alloc(tmem_slot, C::kTmemCols);
@@ -138,73 +182,137 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    if (warp == 0 && lane == 0) {
-        // ------------------------------------------------ scheduler + TMA producer
+    if (warp == 0) {
+        // ------------------------------------------------ scheduler + copy producer
+        // Lane 0 takes tiles and issues every barrier, bulk and TMA operation.  For
+        // routed gate/up tiles with a.row_token set, the whole warp also gathers the
+        // unit's token rows straight from x into the stage (stored with the 128-byte
+        // swizzle, loaded one k-step ahead), so no permuted copy of x is needed.
+        // Every stage's full barrier takes two arrivals: the expect-tx arrival and a
+        // completion arrival once this warp has written or issued everything.
         const uint64_t pol_w = policy_evict_first();   // weights stream through once
         const uint64_t pol_x = policy_evict_last();    // activations are re-read per tile
+        const uint8_t* w_gu = static_cast<const uint8_t*>(a.w_gu);
+        const uint8_t* w_dn = static_cast<const uint8_t*>(a.w_down);
+        const __nv_bfloat16* x_rows = static_cast<const __nv_bfloat16*>(a.x_rows);
         uint32_t it = 0;
         int tc = 0;
         bool ok = true, stuck_pending = a.inject_stuck != 0;
         while (true) {
-            int i = (ok && !error_pending(a.st)) ? atomicAdd(tile_counter, 1) : n_tiles;
+            int i = n_tiles;
+            if (lane == 0 && ok && !error_pending(a.st)) i = atomicAdd(tile_counter, 1);
+            i = __shfl_sync(0xffffffffu, i, 0);
             Tile t = decode_tile(i, n_units, a, mt_gu, mt_dn, BN);
             const int r = tc % kRing;
-            if (!mbar_wait(&tempty[r], ((tc / kRing) & 1) ^ 1, a.st, limit)) { ok = false; break; }
-            ring[r] = t;
-            mbar_arrive(&tfull[r]);
+            int w_ok = 1;
+            if (lane == 0) {
+                w_ok = mbar_wait(&tempty[r], ((tc / kRing) & 1) ^ 1, a.st, limit);
+                if (w_ok) { ring[r] = t; mbar_arrive(&tfull[r]); }
+            }
+            if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
             ++tc;
             if (t.phase < 0) break;
-            if (t.phase == 1 && (a.phases & 1)) {
-                // dependency: the unit's gate/up tiles must have published their h rows
-                const int target = mt_gu + (stuck_pending ? 1 : 0);
-                stuck_pending = false;
-                const int* flag = done + t.unit;
-                if (ld_acquire_gpu(flag) < target) {
-                    const uint64_t t0 = globaltimer_ns();
-                    while (ld_acquire_gpu(flag) < target) {
-                        __nanosleep(64);
-                        if (globaltimer_ns() - t0 > limit) {
-                            report_error(a.st, kErrTimeout);
-                            ok = false;     // finish this tile (output invalid), take no more
-                            break;
-                        }
+            const bool gather = BN <= 32 && t.phase == 0 && a.row_token != nullptr;
+            const int nb16 = (t.n_len + kBoxRows - 1) / kBoxRows;
+            const int KB = t.phase == 0 ? kb_gu : kb_dn;
+            const uint32_t a_bytes = 2 * kABytes;     // a tile pair per k-step
+            const uint32_t bytes = a_bytes + (gather ? 0 : nb16 * kBoxBytes);
+            const uint8_t* a_src =
+                t.phase == 0 ? w_gu + (size_t)(t.expert * mt_gu + t.mt) * kb_gu * a_bytes
+                : t.phase == 1 ? w_dn + (size_t)(t.expert * mt_dn + t.mt) * kb_dn * a_bytes
+                               : w_gu + (size_t)t.mt * kb_dn * a_bytes;   // packed W_r
+            const CUtensorMap* bmap = t.phase == 1 ? &maps.b_h : &maps.b_x;
+            // gather mode: lane covers (row, 16-byte chunk) pairs p = lane + 32 j
+            const __nv_bfloat16* src_row[8];
+            uint4 nx[8];
+            if (gather) {
+                const int my_tok = lane < t.n_len ? a.row_token[t.row_start + lane] : 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int p = lane + 32 * j, rr = p >> 3, cc = p & 7;
+                    const int tok = __shfl_sync(0xffffffffu, my_tok, rr);
+                    src_row[j] = rr < t.n_len ? x_rows + (size_t)tok * a.H + cc * 8 : nullptr;
+                    if (src_row[j]) nx[j] = *reinterpret_cast<const uint4*>(src_row[j]);
+                }
+            }
+            // Down tiles of a fused launch first stream their weights (independent of h),
+            // then wait until the unit's gate/up tiles have published h, then load h rows.
+            const bool gated = t.phase == 1 && fused;
+            const int pre = gated ? min(KB, C::kStages) : 0;
+            int fail = 0;
+            for (int kb = 0; kb < pre; ++kb) {
+                const uint32_t q = it + kb;
+                const int s = q % C::kStages;
+                if (lane == 0) {
+                    if (!mbar_wait(&empty[s], ((q / C::kStages) & 1) ^ 1, a.st, limit)) fail = 1;
+                    else {
+                        mbar_arrive_expect_tx(&full[s], bytes);
+                        bulk_load(smem + s * C::kStageBytes, a_src + (size_t)kb * a_bytes, a_bytes,
+                                  &full[s], pol_w);
                     }
                 }
-                fence_proxy_async_global();
+                if (__shfl_sync(0xffffffffu, fail, 0)) break;
             }
-            const int nb16 = (t.n_len + kBoxRows - 1) / kBoxRows;
-            const int KB = (t.phase == 0 ? a.H : a.I) / kBK;
-            const uint32_t bytes = (t.phase == 0 ? 2 : 1) * kABytes + nb16 * kBoxBytes;
-            bool fail = false;
-            for (int kb = 0; kb < KB; ++kb, ++it) {
-                const int s = it % C::kStages;
-                if (!mbar_wait(&empty[s], ((it / C::kStages) & 1) ^ 1, a.st, limit)) {
-                    fail = true;
-                    break;
+            if (__shfl_sync(0xffffffffu, fail, 0)) { ok = false; break; }
+            if (gated) {
+                if (lane == 0) {
+                    const int target = mt_gu + (stuck_pending ? 1 : 0);
+                    if (!wait_count(done + t.unit, target, a)) ok = false;   // finish the tile anyway
+                    fence_proxy_async_global();
+                    for (int kb = 0; kb < pre; ++kb) {
+                        const int s = (it + kb) % C::kStages;
+                        uint8_t* B = smem + s * C::kStageBytes + 2 * kABytes;
+                        for (int j = 0; j < nb16; ++j)
+                            tma_load_2d(B + j * kBoxBytes, bmap, &full[s], kb * kBK,
+                                        t.row_start + j * kBoxRows, pol_x);
+                        mbar_arrive(&full[s]);
+                    }
                 }
+                stuck_pending = false;
+                ok = __shfl_sync(0xffffffffu, (int)ok, 0);
+                it += pre;
+            }
+            for (int kb = pre; kb < KB; ++kb, ++it) {
+                const int s = it % C::kStages;
                 uint8_t* A0 = smem + s * C::kStageBytes;
                 uint8_t* B = A0 + 2 * kABytes;
-                mbar_arrive_expect_tx(&full[s], bytes);
-                if (t.phase == 0) {
-                    const int row = t.expert * a.I + t.mt * kBM;
-                    tma_load_2d(A0, &maps.a_gate, &full[s], kb * kBK, row, pol_w);
-                    tma_load_2d(A0 + kABytes, &maps.a_up, &full[s], kb * kBK, row, pol_w);
-                    for (int j = 0; j < nb16; ++j)
-                        tma_load_2d(B + j * kBoxBytes, &maps.b_x, &full[s], kb * kBK,
-                                    t.row_start + j * kBoxRows, pol_x);
-                } else {
-                    const int row = t.expert * a.H + t.mt * kBM;
-                    tma_load_2d(A0, &maps.a_down, &full[s], kb * kBK, row, pol_w);
-                    for (int j = 0; j < nb16; ++j)
-                        tma_load_2d(B + j * kBoxBytes, &maps.b_h, &full[s], kb * kBK,
-                                    t.row_start + j * kBoxRows, pol_x);
+                if (lane == 0) {
+                    if (!mbar_wait(&empty[s], ((it / C::kStages) & 1) ^ 1, a.st, limit)) fail = 1;
+                    else {
+                        mbar_arrive_expect_tx(&full[s], bytes);
+                        bulk_load(A0, a_src + (size_t)kb * a_bytes, a_bytes, &full[s], pol_w);
+                        if (!gather)
+                            for (int j = 0; j < nb16; ++j)
+                                tma_load_2d(B + j * kBoxBytes, bmap, &full[s], kb * kBK,
+                                            t.row_start + j * kBoxRows, pol_x);
+                    }
                 }
+                if (__shfl_sync(0xffffffffu, fail, 0)) break;
+                if (gather) {
+                    // rows of this k-step into the stage, then the next k-step's loads
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int p = lane + 32 * j, rr = p >> 3, cc = p & 7;
+                        if (src_row[j])
+                            *reinterpret_cast<uint4*>(B + rr * 128 + ((cc ^ (rr & 7)) << 4)) = nx[j];
+                    }
+                    if (kb + 1 < KB) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            if (src_row[j])
+                                nx[j] = *reinterpret_cast<const uint4*>(src_row[j] + (kb + 1) * kBK);
+                    }
+                    fence_proxy_async_smem();     // generic stores -> tensor-core reads
+                    __syncwarp();
+                }
+                if (lane == 0) mbar_arrive(&full[s]);
             }
-            if (fail) { ok = false; break; }
+            if (__shfl_sync(0xffffffffu, fail, 0)) { ok = false; break; }
         }
         // drain: copies still in flight must land before the CTA exits
-        for (uint32_t q = (it > (uint32_t)C::kStages ? it - C::kStages : 0); q < it; ++q)
-            mbar_wait(&full[q % C::kStages], (q / C::kStages) & 1, a.st, kDrainLimitNs);
+        if (lane == 0)
+            for (uint32_t q = (it > (uint32_t)C::kStages ? it - C::kStages : 0); q < it; ++q)
+                mbar_wait(&full[q % C::kStages], (q / C::kStages) & 1, a.st, kDrainLimitNs);
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------ MMA issuer
         uint32_t it = 0;
@@ -223,7 +331,7 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
             const uint32_t idesc = idesc_bf16_f32(kBM, N);
             const uint32_t d_gate = tmem_base + acc * 2 * BN;
             const uint32_t d_up = d_gate + BN;
-            const int KB = (t.phase == 0 ? a.H : a.I) / kBK;
+            const int KB = t.phase == 0 ? kb_gu : kb_dn;
             bool fail = false;
             for (int kb = 0; kb < KB; ++kb, ++it) {
                 const int s = it % C::kStages;
@@ -236,9 +344,9 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
                 for (int kk = 0; kk < kBK / 16; ++kk) {
                     const uint64_t bd = smem_desc_sw128(b0 + kk * 32);
                     const uint32_t accum = (kb | kk) != 0;
+                    // gate/up: (gate, up) panels; down: two 128-row output blocks
                     tc_mma_bf16(d_gate, smem_desc_sw128(a0 + kk * 32), bd, idesc, accum);
-                    if (t.phase == 0)
-                        tc_mma_bf16(d_up, smem_desc_sw128(a1 + kk * 32), bd, idesc, accum);
+                    tc_mma_bf16(d_up, smem_desc_sw128(a1 + kk * 32), bd, idesc, accum);
                 }
                 tc_commit(&empty[s]);   // frees the stage once these MMAs have read it
             }
@@ -250,7 +358,13 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
         mbar_wait(drainbar, 0, a.st, kDrainLimitNs);
     } else if (warp >= 2) {
         // ------------------------------------------------ epilogue (TMEM -> bf16 rows)
-        const int q = warp & 3;            // TMEM lanes 32q..32q+31 belong to this warp
+        // Warp pairs (q, q + 4) share TMEM lanes 32q..32q+31 and take alternate
+        // 16-column chunks.  A chunk (32 features x 16 rows) is transposed through
+        // shared memory so that each store writes 16 contiguous bytes of a row.
+        const int ew = warp - 2;
+        const int q = warp & 3;
+        const int half = ew >> 2;
+        __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(epi_smem + ew * kEpiStage);
         __nv_bfloat16* hbuf = static_cast<__nv_bfloat16*>(a.hbuf);
         __nv_bfloat16* outb = static_cast<__nv_bfloat16*>(a.out);
         int tc = 0, ac = 0, pub = 0;
@@ -267,46 +381,74 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
             tc_fence_after();
             const uint32_t tg = tmem_base + acc * 2 * BN + (static_cast<uint32_t>(q * 32) << 16);
             const uint32_t tu = tg + BN;
-            const int f = t.mt * kBM + q * 32 + lane;
             const int nc = (t.n_len + 15) / 16;
-            if (t.phase == 0) {
-                __nv_bfloat16* dst = hbuf + (size_t)t.row_start * a.I + f;
-                for (int c = 0; c < nc; ++c) {
-                    float g[16], u[16];
-                    tmem_ld16(tg + c * 16, g);
-                    tmem_ld16(tu + c * 16, u);
-                    tmem_wait_ld();
+            // gate/up: h[rows][mt*128 + 32q + lane] = SiLU(gate) * up
+            // down:    out[rows][mt*256 + p*128 + 32q + lane] = panel p, p = 0, 1
+            if (t.phase == 2) {
+                // router logits: logits[rows][256 mt + 128 p + 32 q + lane], fp32
+                const int e0 = t.mt * 2 * kBM + q * 32 + lane;
+                float* lg = a.logits + (size_t)t.row_start * a.I;
+                for (int c = half; c < nc; c += 2) {
+                    for (int p = 0; p < 2; ++p) {
+                        float v[16];
+                        tmem_ld16((p ? tu : tg) + c * 16, v);
+                        tmem_wait_ld();
+                        const int e = e0 + p * kBM;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int n = c * 16 + j;
-                        if (n < t.n_len)
-                            dst[(size_t)n * a.I] = __float2bfloat16_rn(silu_fast(g[j]) * u[j]);
+                        for (int j = 0; j < 16; ++j)
+                            if (c * 16 + j < t.n_len && e < a.I) lg[(size_t)(c * 16 + j) * a.I + e] = v[j];
                     }
                 }
-            } else {
-                __nv_bfloat16* dst = outb + (size_t)t.row_start * a.H + f;
-                for (int c = 0; c < nc; ++c) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&accempty[acc]);
+                ++ac;
+                continue;
+            }
+            const int ld = t.phase == 0 ? a.I : a.H;
+            const int col0 = t.phase == 0 ? t.mt * kBM : t.mt * 2 * kBM;
+            const int panels = t.phase == 0 ? 1 : (col0 + kBM < a.H ? 2 : 1);
+            __nv_bfloat16* dst = (t.phase == 0 ? hbuf : outb) + (size_t)t.row_start * ld + col0 +
+                                 q * 32;
+            for (int c = half; c < nc; c += 2) {
+                for (int p = 0; p < panels; ++p) {
                     float v[16];
-                    tmem_ld16(tg + c * 16, v);
-                    tmem_wait_ld();
+                    if (t.phase == 0) {
+                        float u[16];
+                        tmem_ld16(tg + c * 16, v);
+                        tmem_ld16(tu + c * 16, u);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int n = c * 16 + j;
-                        if (n < t.n_len) dst[(size_t)n * a.H] = __float2bfloat16_rn(v[j]);
+                        for (int j = 0; j < 16; ++j) v[j] = silu_fast(v[j]) * u[j];
+                    } else {
+                        tmem_ld16((p ? tu : tg) + c * 16, v);
+                        tmem_wait_ld();
                     }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) stage[j * 32 + lane] = __float2bfloat16_rn(v[j]);
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const int vid = lane + 32 * i, row = vid >> 2, seg = vid & 3;
+                        if (c * 16 + row < t.n_len)
+                            *reinterpret_cast<uint4*>(dst + (size_t)(c * 16 + row) * ld + p * kBM +
+                                                      seg * 8) =
+                                *reinterpret_cast<const uint4*>(stage + row * 32 + seg * 8);
+                    }
+                    __syncwarp();
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&accempty[acc]);
             ++ac;
-            if (t.phase == 0 && (a.phases & 2)) {
+            if (t.phase == 0 && fused) {
                 // publish this unit's h rows to the down tiles (other CTAs read them by TMA)
                 __threadfence();
                 fence_proxy_async_global();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(pubbar);
-                if (warp == 2 && lane == 0) {
+                if (ew == 0 && lane == 0) {
                     if (mbar_wait(pubbar, pub & 1, a.st, limit)) red_release_gpu_add(done + t.unit, 1);
                 }
                 ++pub;
@@ -347,6 +489,12 @@ tc_shared_expert_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
 }
 
 template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_router_logits_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
+    tc_experts_body<BN>(maps, a);
+}
+
+template <int BN>
 cudaError_t launch_width(const TcMaps& maps, const TcArgs& a, int grid, cudaStream_t s) {
     static bool configured = false;   // per process; the attribute is per function
     if (!configured) {
@@ -357,10 +505,16 @@ cudaError_t launch_width(const TcMaps& maps, const TcArgs& a, int grid, cudaStre
             e = cudaFuncSetAttribute(tc_shared_expert_kernel<BN>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      TcCfg<BN>::kSmem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(tc_router_logits_kernel<BN>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     TcCfg<BN>::kSmem);
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    if (a.dense_T > 0)
+    if (a.phases == 4)
+        tc_router_logits_kernel<BN><<<grid, kThreads, TcCfg<BN>::kSmem, s>>>(maps, a);
+    else if (a.dense_T > 0)
         tc_shared_expert_kernel<BN><<<grid, kThreads, TcCfg<BN>::kSmem, s>>>(maps, a);
     else
         tc_routed_experts_kernel<BN><<<grid, kThreads, TcCfg<BN>::kSmem, s>>>(maps, a);
@@ -376,7 +530,7 @@ int tc_smem_bytes(int width) {
 cudaError_t launch_tc_experts(const TcMaps& maps, const TcArgs& a, int width, int grid,
                               cudaStream_t s) {
     if (grid <= 0) return cudaSuccess;
-    if (a.H % kBM || a.I % kBM) return cudaErrorInvalidValue;
+    if (a.H % kBM || a.I % kBM) return cudaErrorInvalidValue;   // I, H multiples of 128
     if (width == 32) return launch_width<32>(maps, a, grid, s);
     if (width == 256) return launch_width<256>(maps, a, grid, s);
     return cudaErrorInvalidValue;

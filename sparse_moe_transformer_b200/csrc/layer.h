@@ -35,7 +35,7 @@ struct RouteBufs {
     float* logits;        // [T][E] fp32 scratch (multi-CTA router)
     int32_t* topk_idx;    // [T][k]
     float* topk_w;        // [T][k]
-    int32_t* block_hist;  // [nblocks][E]
+    int32_t* block_hist;  // [nblocks][E] selections per routing block (zeroed by the scan)
     int32_t* block_off;   // [nblocks][E] exclusive prefix over blocks
     int32_t* counts;      // [E]
     int32_t* offsets;     // [E+1]
@@ -44,19 +44,24 @@ struct RouteBufs {
     int32_t* token_slot;  // [T*k]  permuted row of (t, j)
     int32_t* slot_token;  // [T*k]  token of permuted row
     int32_t* slot_expert; // [T*k]  expert of permuted row
-    int32_t* tickets;     // [nblocks + 1] arrival counters (self-resetting)
+    int32_t* tickets;     // [T / 8 + 1] arrival counters (self-resetting)
 };
 
 // ---------------------------------------------------------------- launchers
 // Router: logits (fp32 accumulate), optional fused pre-RMSNorm, Top-k with the
 // lower-index tie rule, renormalised weights, per-block histograms and (when
-// do_scan) the global scan, expert offsets and the GEMM unit list.
+// do_scan) the global scan, expert offsets and the GEMM unit list.  With
+// select_only the logits already sit in rb.logits (tensor-core router).
+// With permute and a single routing block (T <= tb) the last CTA also performs
+// the permutation (what launch_permute would do; the row copy only if xp != null).
 cudaError_t launch_router(int dtype, const void* x, const void* w_router, const void* rms_w,
-                          float rms_eps, void* x_norm, const Dims& d, int T, int tb,
-                          const RouteBufs& rb, int do_scan, int unit_width, int max_units,
-                          const DeviceStatus& st, cudaStream_t s);
+                          float rms_eps, void* x_norm, int permute, void* xp, const Dims& d,
+                          int T, int tb, const RouteBufs& rb, int do_scan, int unit_width,
+                          int max_units, int select_only, const DeviceStatus& st,
+                          cudaStream_t s);
 
-// Gather token rows into expert-contiguous order; fills token_slot / slot_token.
+// Expert-contiguous order of the token rows: fills token_slot / slot_token /
+// slot_expert, and gathers the rows into xp unless xp is null.
 cudaError_t launch_permute(int dtype, const void* x_in, void* xp, const Dims& d, int T, int tb,
                            const RouteBufs& rb, cudaStream_t s);
 
@@ -65,23 +70,64 @@ cudaError_t launch_combine(int dtype, const void* o, const void* shared_out, con
                            void* y, const float* topk_w, const int32_t* token_slot,
                            const Dims& d, int T, cudaStream_t s);
 
+// Tile-contiguous weight layout of the tensor-core path.  A weight matrix
+// [E][R][C] is cut into 128-row x 64-column tiles, each stored as the exact
+// 16 KB image the tensor core reads from shared memory: 128 rows of 128 bytes
+// whose 16-byte chunks are permuted by the 128-byte swizzle (chunk c of row r
+// stored at chunk c ^ (r % 8)).  Tiles come in pairs that one contiguous 32 KB
+// bulk copy moves together:
+//   gate/up: pair (e, mt, kb) = gate tile (e, mt, kb), then up tile (e, mt, kb);
+//   down:    pair (e, mt2, kb) = tiles (e, 2 mt2, kb) and (e, 2 mt2 + 1, kb),
+//            i.e. 256 output rows; a missing odd tile is stored as zeros.
+// Pairs are ordered e, then row block, then kb.  Offsets of element (e, row, col):
+__host__ __device__ inline size_t swizzled_in_tile(int row, int col) {
+    const int r = row % 128, c = col % 64;
+    return (size_t)r * 64 + (((c >> 3) ^ (r & 7)) << 3) + (c & 7);
+}
+__host__ __device__ inline size_t packed_gu_offset(int e, int row, int col, int which, int I,
+                                                   int H) {
+    const int MT = I / 128, KB = H / 64;
+    return ((((size_t)e * MT + row / 128) * KB + col / 64) * 2 + which) * 8192 +
+           swizzled_in_tile(row, col);
+}
+__host__ __device__ inline size_t packed_down_offset(int e, int row, int col, int H, int I) {
+    const int MT2 = (H / 128 + 1) / 2, KB = I / 64, mt = row / 128;
+    return ((((size_t)e * MT2 + mt / 2) * KB + col / 64) * 2 + (mt & 1)) * 8192 +
+           swizzled_in_tile(row, col);
+}
+__host__ __device__ inline size_t packed_down_elems(int E, int H, int I) {
+    return (size_t)E * ((H / 128 + 1) / 2) * (I / 64) * 2 * 8192;
+}
+
+// Pack weights into the tile-contiguous layout (bf16): gate/up pairs when
+// src1 != nullptr, else down row-block pairs (dst must be zeroed when R / 128 is odd).
+cudaError_t launch_pack_tiles(const void* src0, const void* src1, void* dst, int E, int R, int C,
+                              cudaStream_t s);
+
 // CUDA-core expert kernels (exact fp32 accumulate; any shape).
 // rows: permuted rows (routed) or tokens (shared, slot_expert == nullptr).
+// packed: weights are in the tile-contiguous layout (gate/up in one buffer).
 cudaError_t launch_simt_gate_up(int dtype, const void* xin, const void* w_gate, const void* w_up,
-                                const int32_t* slot_expert, const int32_t* n_rows_dev,
+                                int packed, const int32_t* slot_expert, const int32_t* n_rows_dev,
                                 int max_rows, int H, int I, void* hbuf, cudaStream_t s);
-cudaError_t launch_simt_down(int dtype, const void* hbuf, const void* w_down,
+cudaError_t launch_simt_down(int dtype, const void* hbuf, const void* w_down, int packed,
                              const int32_t* slot_expert, const int32_t* n_rows_dev, int max_rows,
                              int H, int I, void* out, cudaStream_t s);
 
 // tcgen05 grouped SwiGLU expert GEMM (bf16, fp32 accumulate).
 struct TcMaps {
-    CUtensorMap a_gate, a_up, a_down;   // weights [E*I][H], [E*I][H], [E*H][I]
-    CUtensorMap b_x, b_h;               // activations [rows][H], [rows][I]
+    CUtensorMap b_x, b_h; // activations [rows][H], [rows][I], 16-row boxes, 128-byte swizzle
 };
 struct TcArgs {
-    int H, I;
-    int phases;          // 1: gate/up, 2: down, 3: both in one launch with dependencies
+    const void* w_gu;     // packed gate/up tiles (see packed_gu_offset); router: packed W_r
+    const void* w_down;   // packed down tiles (see packed_down_offset)
+    int H, I;             // router launch: I = number of experts E
+    int phases;          // 1: gate/up, 2: down, 3: both in one launch with dependencies,
+                         // 4: router logits (dense over dense_T tokens, fp32 into `logits`)
+    float* logits;       // [dense_T][I] fp32, router launch only
+    const void* x_rows;       // gather mode: token rows [T][H] bf16 (x or its normalised copy)
+    const int32_t* row_token; // non-null: routed gate/up tiles gather row r from x_rows
+                              // [row_token[r]] instead of loading permuted rows by TMA
     int dense_T;         // >0: units are consecutive row runs over dense_T rows (shared expert)
     int unit_width;      // tile width the units were built with
     const Unit* units;

@@ -9,7 +9,7 @@
 #include <algorithm>
 #include <vector>
 
-#include "../../include/moe.h"
+#include "moe.h"
 #include "layer.h"
 
 using namespace moe;
@@ -85,7 +85,8 @@ moe_status make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
     return MOE_OK;
 }
 
-constexpr int kRouteBlock = 16;      // tokens per router CTA / permutation block
+constexpr int kRouteBlock = 16;      // routing block with CUDA-core logits (T < 256)
+constexpr int kRouteBlockWide = 64;  // routing block after tensor-core logits
 constexpr int kNarrow = 32, kWide = 256;
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -103,6 +104,7 @@ struct moe_layer {
     // owned weight copies
     void *w_router = nullptr, *w_gate = nullptr, *w_up = nullptr, *w_down = nullptr;
     void *ws_gate = nullptr, *ws_up = nullptr, *ws_down = nullptr, *rms_w = nullptr;
+    void* w_router_packed = nullptr;   // tensor-core router (E % 128 == 0, no pre-norm)
     // workspace
     int max_T = 0;
     int max_units = 0;
@@ -111,7 +113,7 @@ struct moe_layer {
     void *x_norm = nullptr, *xp = nullptr, *hbuf = nullptr, *obuf = nullptr;
     void *hs = nullptr, *sbuf = nullptr;
     void *x_stage = nullptr, *r_stage = nullptr, *y_stage = nullptr;
-    int32_t *sync_routed = nullptr, *sync_shared = nullptr;
+    int32_t *sync_routed = nullptr, *sync_shared = nullptr, *sync_router = nullptr;
     TcMaps routed_maps{}, shared_maps{};
     // status words
     int* err_dev = nullptr;
@@ -140,6 +142,17 @@ moe_status copy_weight(void** dst, const void* src, size_t bytes) {
     if (!bytes) return MOE_OK;
     CUDA_TRY(cudaMalloc(dst, bytes));
     CUDA_TRY(cudaMemcpy(*dst, src, bytes, cudaMemcpyDeviceToDevice));
+    return MOE_OK;
+}
+
+// Allocate and fill a tile-contiguous copy of one or two expert-major matrices
+// (see packed_gu_offset / packed_down_offset).
+moe_status pack_weight(void** dst, const void* src0, const void* src1, int E, int R, int C) {
+    const size_t bytes = src1 ? (size_t)E * R * C * 2 * 2 : packed_down_elems(E, R, C) * 2;
+    CUDA_TRY(cudaMalloc(dst, bytes));
+    CUDA_TRY(cudaMemset(*dst, 0, bytes));
+    CUDA_TRY(launch_pack_tiles(src0, src1, *dst, E, R, C, 0));
+    CUDA_TRY(cudaStreamSynchronize(0));
     return MOE_OK;
 }
 
@@ -260,13 +273,25 @@ moe_status moe_create(const moe_config* cfg, int device, const void* w_router, c
     moe_status st = MOE_OK;
     auto chk = [&](moe_status s) { if (st == MOE_OK) st = s; };
     chk(copy_weight(&h->w_router, w_router, E * H * es));
-    chk(copy_weight(&h->w_gate, w_gate, E * I * H * es));
-    chk(copy_weight(&h->w_up, w_up, E * I * H * es));
-    chk(copy_weight(&h->w_down, w_down, E * H * I * es));
-    if (Is) {
-        chk(copy_weight(&h->ws_gate, ws_gate, Is * H * es));
-        chk(copy_weight(&h->ws_up, ws_up, Is * H * es));
-        chk(copy_weight(&h->ws_down, ws_down, H * Is * es));
+    if (h->tc_ok) {
+        // tile-contiguous copies: gate/up interleaved in w_gate, w_up unused
+        chk(pack_weight(&h->w_gate, w_gate, w_up, (int)E, (int)I, (int)H));
+        chk(pack_weight(&h->w_down, w_down, nullptr, (int)E, (int)H, (int)I));
+        if (E % 128 == 0 && !rms_weight)
+            chk(pack_weight(&h->w_router_packed, w_router, nullptr, 1, (int)E, (int)H));
+        if (Is) {
+            chk(pack_weight(&h->ws_gate, ws_gate, ws_up, 1, (int)Is, (int)H));
+            chk(pack_weight(&h->ws_down, ws_down, nullptr, 1, (int)H, (int)Is));
+        }
+    } else {
+        chk(copy_weight(&h->w_gate, w_gate, E * I * H * es));
+        chk(copy_weight(&h->w_up, w_up, E * I * H * es));
+        chk(copy_weight(&h->w_down, w_down, E * H * I * es));
+        if (Is) {
+            chk(copy_weight(&h->ws_gate, ws_gate, Is * H * es));
+            chk(copy_weight(&h->ws_up, ws_up, Is * H * es));
+            chk(copy_weight(&h->ws_down, ws_down, H * Is * es));
+        }
     }
     if (rms_weight) chk(copy_weight(&h->rms_w, rms_weight, H * es));
     if (st == MOE_OK) {
@@ -281,16 +306,6 @@ moe_status moe_create(const moe_config* cfg, int device, const void* w_router, c
         if (e != cudaSuccess)
             chk(fail(e == cudaErrorMemoryAllocation ? MOE_ERR_OOM : MOE_ERR_CUDA, "create: %s",
                      cudaGetErrorString(e)));
-    }
-    if (st == MOE_OK && h->tc_ok) {
-        chk(make_map(&h->routed_maps.a_gate, h->w_gate, E * I, H, 128));
-        chk(make_map(&h->routed_maps.a_up, h->w_up, E * I, H, 128));
-        chk(make_map(&h->routed_maps.a_down, h->w_down, E * H, I, 128));
-        if (Is) {
-            chk(make_map(&h->shared_maps.a_gate, h->ws_gate, Is, H, 128));
-            chk(make_map(&h->shared_maps.a_up, h->ws_up, Is, H, 128));
-            chk(make_map(&h->shared_maps.a_down, h->ws_down, H, Is, 128));
-        }
     }
     if (st != MOE_OK) {
         char keep[sizeof g_err];
@@ -329,9 +344,10 @@ moe_status moe_reserve(moe_handle h, int max_tokens) {
         {(void**)&h->rb.token_slot, S * 4},
         {(void**)&h->rb.slot_token, S * 4},
         {(void**)&h->rb.slot_expert, S * 4},
-        {(void**)&h->rb.tickets, (nblocks + 1) * 4},
+        {(void**)&h->rb.tickets, ((T + 7) / 8 + 1) * 4},        // CTA groups of >= 8 tokens
         {(void**)&h->sync_routed, (2 + (size_t)max_units) * 4},
         {(void**)&h->sync_shared, (2 + (size_t)max_shared_units) * 4},
+        {(void**)&h->sync_router, (2 + (size_t)max_shared_units) * 4},
         {&h->x_norm, h->rms_w ? T * H * es : 0},
         {&h->xp, S * H * es},
         {&h->hbuf, S * I * es},
@@ -373,6 +389,29 @@ int choose_width(const moe_layer* h, int T) {
     return (int64_t)T * h->d.k > (int64_t)16 * h->d.E ? kWide : kNarrow;
 }
 
+// Tensor-core router logits for large T: W_r (packed) x tokens, fp32 into rb.logits.
+bool use_tc_router(const moe_layer* h, int T) {
+    return h->w_router_packed && !h->force_simt && T >= 256;
+}
+
+moe_status run_tc_router(moe_layer* h, const void* x, int T, const RouteBufs& rb,
+                         cudaStream_t s) {
+    const Dims& d = h->d;
+    TcMaps maps{};
+    moe_status st = make_map(&maps.b_x, x, (uint64_t)T, d.H, 16);
+    if (st != MOE_OK) return st;
+    maps.b_h = maps.b_x;
+    TcArgs a{};
+    a.w_gu = h->w_router_packed; a.w_down = nullptr;
+    a.H = d.H; a.I = d.E; a.phases = 4; a.logits = rb.logits;
+    a.dense_T = T; a.unit_width = kNarrow;
+    a.sync = h->sync_router;
+    a.st = h->status(); a.wait_limit_ns = h->wait_limit_ns; a.inject_stuck = 0;
+    const int tiles = (T + kNarrow - 1) / kNarrow * ((d.E / 128 + 1) / 2);
+    CUDA_TRY(launch_tc_experts(maps, a, kNarrow, std::min(tiles, h->num_sms), s));
+    return MOE_OK;
+}
+
 moe_status run_shared(moe_layer* h, const void* x_in, int T, cudaStream_t s) {
     const Dims& d = h->d;
     if (!d.Is) return MOE_OK;
@@ -382,13 +421,14 @@ moe_status run_shared(moe_layer* h, const void* x_in, int T, cudaStream_t s) {
         if (st != MOE_OK) return st;
         const int width = choose_width(h, T);
         TcArgs a{};
+        a.w_gu = h->ws_gate; a.w_down = h->ws_down;
         a.H = d.H; a.I = d.Is; a.phases = h->fuse ? 3 : 1;
         a.dense_T = T; a.unit_width = width;
         a.units = nullptr; a.n_units = nullptr;
         a.sync = h->sync_shared; a.hbuf = h->hs; a.out = h->sbuf;
         a.st = h->status(); a.wait_limit_ns = h->wait_limit_ns; a.inject_stuck = 0;
         const int units = (T + width - 1) / width;
-        const int tiles = units * (d.Is / 128 + d.H / 128);
+        const int tiles = units * (d.Is / 128 + (d.H / 128 + 1) / 2);
         {
             KernelScope ks(h, MOE_KERNEL_SHARED, s);
             CUDA_TRY(launch_tc_experts(maps, a, width, std::min(tiles, h->num_sms), s));
@@ -401,12 +441,12 @@ moe_status run_shared(moe_layer* h, const void* x_in, int T, cudaStream_t s) {
     } else {
         {
             KernelScope ks(h, MOE_KERNEL_SHARED, s);
-            CUDA_TRY(launch_simt_gate_up(h->dtype, x_in, h->ws_gate, h->ws_up, nullptr, nullptr,
-                                         T, d.H, d.Is, h->hs, s));
+            CUDA_TRY(launch_simt_gate_up(h->dtype, x_in, h->ws_gate, h->ws_up, h->tc_ok, nullptr,
+                                         nullptr, T, d.H, d.Is, h->hs, s));
         }
         KernelScope ks(h, MOE_KERNEL_SHARED, s);
-        CUDA_TRY(launch_simt_down(h->dtype, h->hs, h->ws_down, nullptr, nullptr, T, d.H, d.Is,
-                                  h->sbuf, s));
+        CUDA_TRY(launch_simt_down(h->dtype, h->hs, h->ws_down, h->tc_ok, nullptr, nullptr, T,
+                                  d.H, d.Is, h->sbuf, s));
     }
     return MOE_OK;
 }
@@ -429,10 +469,21 @@ moe_status run_layer(moe_layer* h, const void* x, const void* residual, void* y,
         if (st != MOE_OK) return st;
         CUDA_TRY(cudaEventRecord(h->ev_join, h->s2));
     }
+    const bool tc_route = use_tc_router(h, T);
+    const int tb = tc_route ? kRouteBlockWide : kRouteBlock;
+    const bool fused_permute = T <= tb;      // one routing block: the router permutes it
+    // narrow tensor-core tiles read their token rows from x in place: no permuted copy
+    const bool gather = tc && width == kNarrow;
+    void* xp_copy = gather ? nullptr : h->xp;
     {
         KernelScope ks(h, MOE_KERNEL_ROUTER, s);
-        CUDA_TRY(launch_router(h->dtype, x, h->w_router, h->rms_w, h->cfg.rms_eps, h->x_norm, d,
-                               T, kRouteBlock, rb, 1, width, h->max_units, h->status(), s));
+        if (tc_route) {
+            moe_status st = run_tc_router(h, x, T, rb, s);
+            if (st != MOE_OK) return st;
+        }
+        CUDA_TRY(launch_router(h->dtype, x, h->w_router, h->rms_w, h->cfg.rms_eps, h->x_norm,
+                               fused_permute, xp_copy, d, T, tb, rb, 1, width, h->max_units,
+                               tc_route, h->status(), s));
     }
     if (side && h->rms_w) {      // with a pre-norm it needs the router's normalised x
         CUDA_TRY(cudaEventRecord(h->ev_fork, s));
@@ -441,21 +492,23 @@ moe_status run_layer(moe_layer* h, const void* x, const void* residual, void* y,
         if (st != MOE_OK) return st;
         CUDA_TRY(cudaEventRecord(h->ev_join, h->s2));
     }
-    {
+    if (!fused_permute) {
         KernelScope ks(h, MOE_KERNEL_PERMUTE, s);
-        CUDA_TRY(launch_permute(h->dtype, x_in, h->xp, d, T, kRouteBlock, rb, s));
+        CUDA_TRY(launch_permute(h->dtype, x_in, xp_copy, d, T, tb, rb, s));
     }
     const int S = T * d.k;
     if (tc) {
         TcArgs a{};
+        a.w_gu = h->w_gate; a.w_down = h->w_down;
         a.H = d.H; a.I = d.I; a.phases = h->fuse ? 3 : 1;
         a.dense_T = 0; a.unit_width = width;
         a.units = rb.units; a.n_units = rb.n_units;
+        a.x_rows = x_in; a.row_token = gather ? rb.slot_token : nullptr;
         a.sync = h->sync_routed; a.hbuf = h->hbuf; a.out = h->obuf;
         a.st = h->status(); a.wait_limit_ns = h->wait_limit_ns;
         a.inject_stuck = h->inject_stuck && h->fuse;
         const int max_units = std::min(h->max_units, (S + width - 1) / width + d.E);
-        const int tiles = max_units * (d.I / 128 + d.H / 128);
+        const int tiles = max_units * (d.I / 128 + (d.H / 128 + 1) / 2);
         const int grid = std::min(tiles, h->num_sms);
         {
             KernelScope ks(h, MOE_KERNEL_EXPERTS, s);
@@ -471,12 +524,12 @@ moe_status run_layer(moe_layer* h, const void* x, const void* residual, void* y,
         const int32_t* n_rows = rb.offsets + d.E;
         {
             KernelScope ks(h, MOE_KERNEL_EXPERTS, s);
-            CUDA_TRY(launch_simt_gate_up(h->dtype, h->xp, h->w_gate, h->w_up, rb.slot_expert,
-                                         n_rows, S, d.H, d.I, h->hbuf, s));
+            CUDA_TRY(launch_simt_gate_up(h->dtype, h->xp, h->w_gate, h->w_up, h->tc_ok,
+                                         rb.slot_expert, n_rows, S, d.H, d.I, h->hbuf, s));
         }
         KernelScope ks(h, MOE_KERNEL_EXPERTS, s);
-        CUDA_TRY(launch_simt_down(h->dtype, h->hbuf, h->w_down, rb.slot_expert, n_rows, S, d.H,
-                                  d.I, h->obuf, s));
+        CUDA_TRY(launch_simt_down(h->dtype, h->hbuf, h->w_down, h->tc_ok, rb.slot_expert, n_rows,
+                                  S, d.H, d.I, h->obuf, s));
     }
     if (d.Is > 0) {
         if (side) {
@@ -505,6 +558,7 @@ moe_status moe_route(moe_handle h, const void* x, int T, int32_t* topk_idx, floa
     if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T < 0");
     if (T == 0) return MOE_OK;
     if (!x || !topk_idx || !topk_w) return fail(MOE_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(x)) return fail(MOE_ERR_INVALID_ARG, "x must be 16-byte aligned");
     if (T > h->max_T) return fail(MOE_ERR_INVALID_ARG, "T=%d exceeds reserved %d", T, h->max_T);
     moe_status pe = pending_device_error(h);
     if (pe != MOE_OK) return pe;
@@ -513,9 +567,14 @@ moe_status moe_route(moe_handle h, const void* x, int T, int32_t* topk_idx, floa
     rb.topk_idx = topk_idx;
     rb.topk_w = topk_w;
     KernelScope ks(h, MOE_KERNEL_ROUTER, (cudaStream_t)stream);
-    CUDA_TRY(launch_router(h->dtype, x, h->w_router, h->rms_w, h->cfg.rms_eps, nullptr, h->d, T,
-                           kRouteBlock, rb, 0, kNarrow, h->max_units, h->status(),
-                           (cudaStream_t)stream));
+    if (use_tc_router(h, T)) {
+        moe_status st = run_tc_router(h, x, T, rb, (cudaStream_t)stream);
+        if (st != MOE_OK) return st;
+    }
+    const bool tc_route = use_tc_router(h, T);
+    CUDA_TRY(launch_router(h->dtype, x, h->w_router, h->rms_w, h->cfg.rms_eps, nullptr, 0,
+                           nullptr, h->d, T, tc_route ? kRouteBlockWide : kRouteBlock, rb, 0,
+                           kNarrow, h->max_units, tc_route, h->status(), (cudaStream_t)stream));
     return MOE_OK;
 }
 
@@ -632,8 +691,8 @@ moe_status moe_destroy(moe_handle h) {
     for (auto& p : h->pending) { cudaEventDestroy(p.a); cudaEventDestroy(p.b); }
     for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
     free_workspace(h);
-    void* bufs[] = {h->w_router, h->w_gate, h->w_up, h->w_down, h->ws_gate,
-                    h->ws_up,    h->ws_down, h->rms_w, h->err_dev};
+    void* bufs[] = {h->w_router, h->w_gate, h->w_up,  h->w_down,  h->ws_gate,
+                    h->ws_up,    h->ws_down, h->rms_w, h->err_dev, h->w_router_packed};
     for (void* p : bufs)
         if (p) cudaFree(p);
     if (h->err_host) cudaFreeHost(h->err_host);

@@ -8,8 +8,15 @@
 // only the k selected logits.  Optional pre-RMSNorm: "rmsnorm" helper of the lab
 // page, section [3C], x / sqrt(mean(x^2) + eps) * g, applied in fp32 before the
 // logits (the router never sees a rounded normalised input).
+//
+// These kernels run once per layer call on little data, so they are written to
+// be latency-lean: short rolled loops (the code is fetched cold on every
+// launch), loads issued together, and block-wide parallel scans instead of
+// single-thread loops.
 #include <cuda_bf16.h>
 #include <stdint.h>
+
+#include <algorithm>
 
 #include "device.cuh"
 #include "layer.h"
@@ -17,270 +24,447 @@
 namespace moe {
 namespace {
 
-constexpr int kRouterThreads = 256;
-constexpr int kEG = 16;        // experts per router CTA
-constexpr int kMaxTB = 16;     // tokens per router CTA (= routing block)
-constexpr int kKC = 128;       // K chunk staged in shared memory
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kEG = 2;              // experts per logits CTA: 4 warps per expert
+constexpr int kMaxTB = 16;          // tokens per logits CTA
 constexpr int kMaxE = 1024;
 constexpr int kMaxK = 16;
+constexpr int kChunk = 32;          // routing blocks per scan chunk
 
-// "a before b" in the Top-k order: larger logit first, ties to the lower index.
-__device__ __forceinline__ bool before(float va, int ia, float vb, int ib) {
-    return va > vb || (va == vb && ia < ib);
+// VEC consecutive elements as fp32 (VEC * sizeof(T) == 16: one vector load).
+template <typename T, int VEC>
+__device__ __forceinline__ void load_vec(const T* p, float (&v)[VEC]) {
+    if constexpr (VEC * sizeof(T) == 16) {
+        uint4 raw = *reinterpret_cast<const uint4*>(p);
+        const T* e = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) v[i] = to_f32(e[i]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) v[i] = to_f32(p[i]);
+    }
 }
 
-template <typename Tin>
-__global__ void __launch_bounds__(kRouterThreads)
-router_kernel(const Tin* __restrict__ x, const Tin* __restrict__ w_router,
-              const Tin* __restrict__ rms_w, float rms_eps, Tin* __restrict__ x_norm, Dims d,
-              int T, int tb, RouteBufs rb, int do_scan, int unit_width, int max_units,
-              DeviceStatus st) {
-    __shared__ float xs[kMaxTB][kKC + 1];
-    __shared__ float ws[kEG][kKC + 1];
-    __shared__ float inv_rms[kMaxTB];
-    __shared__ int hist[kMaxE];
-    __shared__ int unit_base[kMaxE + 1];
-    __shared__ int s_flag;
-
+// In-place exclusive scan of v[0..n) (n <= 1024) by all kThreads threads;
+// returns the total.  `tmp` holds kWarps + 1 ints of shared memory.
+__device__ int block_exclusive_scan(int* v, int n, int* tmp) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int H = d.H, E = d.E, k = d.k;
-    const int n_groups = gridDim.x, nblocks = gridDim.y;
-    const int g = blockIdx.x, b = blockIdx.y;
-    const int t0 = b * tb, nt = min(tb, T - t0);
-    const int e0 = g * kEG;
-
-    // ---- pre-RMSNorm scale per token (fp32), one warp per token
-    if (rms_w) {
-        for (int tl = warp; tl < nt; tl += kRouterThreads / 32) {
-            const Tin* row = x + (size_t)(t0 + tl) * H;
-            float ss = 0.f;
-            for (int j = lane; j < H; j += 32) {
-                float v = to_f32(row[j]);
-                ss += v * v;
-            }
+    const int per = (n + kThreads - 1) / kThreads;
+    const int b0 = min(n, tid * per), b1 = min(n, b0 + per);
+    int s = 0;
+    for (int i = b0; i < b1; ++i) s += v[i];
+    int incl = s;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            if (lane == 0) inv_rms[tl] = 1.0f / sqrtf(ss / (float)H + rms_eps);
-        }
-        __syncthreads();
-        if (g == 0 && x_norm) {   // materialise the normalised input for the experts
-            for (int i = tid; i < nt * H; i += kRouterThreads) {
-                int tl = i / H, j = i - tl * H;
-                float v = to_f32(x[(size_t)(t0 + tl) * H + j]) * inv_rms[tl] * to_f32(rms_w[j]);
-                x_norm[(size_t)(t0 + tl) * H + j] = from_f32<Tin>(v);
-            }
-        }
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
     }
-
-    // ---- logits for nt tokens x kEG experts; thread = (token, expert)
-    const int tl_me = tid / kEG, el_me = tid % kEG;
-    float acc = 0.f;
-    for (int kc = 0; kc < H; kc += kKC) {
-        const int kn = min(kKC, H - kc);
-        for (int i = tid; i < kMaxTB * kKC; i += kRouterThreads) {
-            int tl = i / kKC, j = i - tl * kKC;
-            float v = 0.f;
-            if (tl < nt && j < kn) {
-                v = to_f32(x[(size_t)(t0 + tl) * H + kc + j]);
-                if (rms_w) v = v * inv_rms[tl] * to_f32(rms_w[kc + j]);
-            }
-            xs[tl][j] = v;
-        }
-        for (int i = tid; i < kEG * kKC; i += kRouterThreads) {
-            int el = i / kKC, j = i - el * kKC;
-            ws[el][j] = (e0 + el < E && j < kn) ? to_f32(w_router[(size_t)(e0 + el) * H + kc + j])
-                                                : 0.f;
-        }
-        __syncthreads();
-#pragma unroll 8
-        for (int j = 0; j < kKC; ++j) acc = fmaf(xs[tl_me][j], ws[el_me][j], acc);
-        __syncthreads();
-    }
-    if (tl_me < nt && e0 + el_me < E) rb.logits[(size_t)(t0 + tl_me) * E + e0 + el_me] = acc;
-
-    // ---- the last CTA of this token block selects the Top-k
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_flag = (atomicAdd(&rb.tickets[b], 1) == n_groups - 1);
-    __syncthreads();
-    if (!s_flag) return;
-    __threadfence();
-    for (int e = tid; e < E; e += kRouterThreads) hist[e] = 0;
-    __syncthreads();
-
-    for (int tl = warp; tl < nt; tl += kRouterThreads / 32) {
-        const int t = t0 + tl;
-        const float* lrow = rb.logits + (size_t)t * E;
-        uint32_t taken = 0;     // bit i: element lane + 32 i already selected
-        float sel_v[kMaxK];
-        int sel_i[kMaxK];
-        for (int r = 0; r < k; ++r) {
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
-            for (int i = 0; lane + 32 * i < E; ++i) {
-                if (taken & (1u << i)) continue;
-                int e = lane + 32 * i;
-                float v = __ldcg(lrow + e);
-                if (bi == 0x7fffffff || before(v, e, bv, bi)) { bv = v; bi = e; }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (oi != 0x7fffffff && (bi == 0x7fffffff || before(ov, oi, bv, bi))) {
-                    bv = ov; bi = oi;
-                }
-            }
-            if (bi != 0x7fffffff && (bi & 31) == lane) taken |= 1u << (bi >> 5);
-            sel_v[r] = bv;
-            sel_i[r] = bi;
-        }
-        if (lane == 0) {
-            float z = 0.f, ex[kMaxK];
-            for (int r = 0; r < k; ++r) { ex[r] = expf(sel_v[r] - sel_v[0]); z += ex[r]; }
-            for (int r = 0; r < k; ++r) {
-                int e = sel_i[r];
-                if (e < 0 || e >= E) { report_error(st, kErrDeviceCheck); e = 0; }
-                rb.topk_idx[(size_t)t * k + r] = e;
-                rb.topk_w[(size_t)t * k + r] = ex[r] / z;
-                atomicAdd(&hist[e], 1);
-            }
-        }
-    }
-    __syncthreads();
-    for (int e = tid; e < E; e += kRouterThreads) rb.block_hist[(size_t)b * E + e] = hist[e];
-    if (tid == 0) rb.tickets[b] = 0;   // every CTA of this block has arrived
-    if (!do_scan) return;
-
-    // ---- the last token block computes the global scan and the unit list
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_flag = (atomicAdd(&rb.tickets[nblocks], 1) == nblocks - 1);
-    __syncthreads();
-    if (!s_flag) return;
-    __threadfence();
-    for (int e = tid; e < E; e += kRouterThreads) {
-        int run = 0;
-        for (int bb = 0; bb < nblocks; ++bb) {
-            rb.block_off[(size_t)bb * E + e] = run;
-            run += __ldcg(rb.block_hist + (size_t)bb * E + e);
-        }
-        hist[e] = run;
-        rb.counts[e] = run;
-    }
+    if (lane == 31) tmp[warp] = incl;
     __syncthreads();
     if (tid == 0) {
-        int off = 0, nu = 0;
-        for (int e = 0; e < E; ++e) {
-            rb.offsets[e] = off;
-            unit_base[e] = nu;
-            off += hist[e];
-            nu += (hist[e] + unit_width - 1) / unit_width;
-        }
-        rb.offsets[E] = off;
-        unit_base[E] = nu;
-        if (nu > max_units) { report_error(st, kErrDeviceCheck); nu = max_units; }
-        *rb.n_units = nu;
-        rb.tickets[nblocks] = 0;
+        int run = 0;
+        for (int w = 0; w < kWarps; ++w) { const int t = tmp[w]; tmp[w] = run; run += t; }
+        tmp[kWarps] = run;
     }
     __syncthreads();
-    for (int e = tid; e < E; e += kRouterThreads) {
-        int c = hist[e], base = rb.offsets[e];
-        for (int u = 0; u * unit_width < c; ++u) {
-            int idx = unit_base[e] + u;
-            if (idx >= max_units) break;
+    int run = tmp[warp] + incl - s;
+    for (int i = b0; i < b1; ++i) { const int t = v[i]; v[i] = run; run += t; }
+    const int total = tmp[kWarps];
+    __syncthreads();
+    return total;
+}
+
+// Order-preserving map of an fp32 value to uint32 (larger float -> larger key;
+// -0 and +0 map to the same key, so they tie like equal values).
+__device__ __forceinline__ uint32_t order_key(float f) {
+    const uint32_t u = __float_as_uint(f + 0.0f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Top-k of one token (one warp): EPL logits per lane (experts lane + 32 i).
+// Each round: every lane proposes its best unselected expert; the warp takes
+// the largest key (redux.sync max) and, among equal keys, the lowest expert
+// index (redux.sync min) -- the lower-index tie rule.  The selections are
+// counted into the token's routing block (hist = its row, nullable).
+template <int EPL>
+__device__ void warp_topk(const float* lrow, int E, int k, int t, RouteBufs& rb, int* hist,
+                          const DeviceStatus& st) {
+    const int lane = threadIdx.x & 31;
+    float lv[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+        lv[i] = (lane + 32 * i < E) ? __ldcg(lrow + lane + 32 * i) : -INFINITY;
+    uint32_t taken = 0;                 // bit i: element lane + 32 i already selected
+    float vmax = 0.f, z = 0.f, my_v = 0.f;
+    int my_e = -1;
+#pragma unroll 1
+    for (int r = 0; r < k; ++r) {
+        uint32_t bk = 0;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int e = lane + 32 * i;
+            const uint32_t key = order_key(lv[i]);
+            if (e < E && !(taken & (1u << i)) && (bi == 0x7fffffff || key > bk)) { bk = key; bi = e; }
+        }
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, bk);
+        int e_win = (int)__reduce_min_sync(0xffffffffu, (bi != 0x7fffffff && bk == kmax)
+                                                            ? (uint32_t)bi : 0xffffffffu);
+        if (e_win < 0 || e_win >= E) {            // cannot happen for k <= E
+            if (lane == 0) report_error(st, kErrDeviceCheck);
+            e_win = r;
+        }
+        if ((e_win & 31) == lane) taken |= 1u << (e_win >> 5);
+        float bv = 0.f;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) if (lane + 32 * i == e_win) bv = lv[i];
+        bv = __shfl_sync(0xffffffffu, bv, e_win & 31);
+        if (r == 0) vmax = bv;
+        const float ex = expf(bv - vmax);
+        z += ex;
+        if (lane == r) { my_e = e_win; my_v = ex; }   // lane r keeps selection r
+    }
+    if (lane < k) {
+        rb.topk_idx[(size_t)t * k + lane] = my_e;
+        rb.topk_w[(size_t)t * k + lane] = my_v / z;
+        if (hist) atomicAdd(hist + my_e, 1);
+    }
+}
+
+// Permutation of routing block b (tb <= 128 tokens): rows of one expert in token
+// order.  rank = earlier tokens of the block that chose the same expert (from a
+// 128-bit token mask per expert) + earlier blocks' counts.  part / split: this
+// CTA copies every split-th 16-byte vector of the block's rows (no copy when xp is
+// null: bookkeeping only).  `sm` holds E * 4 + tb * k ints of shared memory.
+template <typename Tin>
+__device__ void permute_block(const Tin* __restrict__ x_in, Tin* __restrict__ xp, const Dims& d,
+                              int T, int tb, int b, int part, int split, const RouteBufs& rb,
+                              uint32_t* sm) {
+    const int tid = threadIdx.x;
+    const int E = d.E, k = d.k, H = d.H;
+    const int t0 = b * tb, nt = min(tb, T - t0), pairs = nt * k;
+    uint32_t* bits = sm;
+    int* pos_s = reinterpret_cast<int*>(sm + E * 4);
+    for (int i = tid; i < E * 4; i += blockDim.x) bits[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < pairs; i += blockDim.x) {
+        const int tl = i / k;
+        const int e = __ldcg(rb.topk_idx + (size_t)t0 * k + i);
+        atomicOr(&bits[e * 4 + (tl >> 5)], 1u << (tl & 31));
+    }
+    __syncthreads();
+    for (int i = tid; i < pairs; i += blockDim.x) {
+        const int tl = i / k;
+        const int e = __ldcg(rb.topk_idx + (size_t)t0 * k + i);
+        int rank = __popc(bits[e * 4 + (tl >> 5)] & ((1u << (tl & 31)) - 1u));
+        for (int w = 0; w < (tl >> 5); ++w) rank += __popc(bits[e * 4 + w]);
+        const int pos = __ldcg(rb.offsets + e) + __ldcg(rb.block_off + (size_t)b * E + e) + rank;
+        pos_s[i] = pos;
+        if (part == 0) {
+            rb.token_slot[(size_t)t0 * k + i] = pos;
+            rb.slot_token[pos] = t0 + tl;
+            rb.slot_expert[pos] = e;
+        }
+    }
+    __syncthreads();
+    if (!xp) return;                                       // bookkeeping only
+    if ((H * (int)sizeof(Tin)) % 16 == 0) {
+        const int nv = H * (int)sizeof(Tin) / 16;            // vectors per row
+        const int total = pairs * nv;
+        const int stride = blockDim.x * split;
+#pragma unroll 1
+        for (int q0 = part * blockDim.x + tid; q0 < total; q0 += 8 * stride) {
+            uint4 v[8];
+            int dst[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {                    // eight loads in flight
+                const int q = q0 + u * stride;
+                dst[u] = -1;
+                if (q < total) {
+                    const int i = q / nv, c = q - i * nv;
+                    v[u] = *(reinterpret_cast<const uint4*>(x_in + (size_t)(t0 + i / k) * H) + c);
+                    dst[u] = pos_s[i] * nv + c;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (dst[u] >= 0) reinterpret_cast<uint4*>(xp)[dst[u]] = v[u];
+        }
+    } else {
+        for (int q = part * blockDim.x + tid; q < pairs * H; q += blockDim.x * split) {
+            const int i = q / H, j = q - i * H;
+            xp[(size_t)pos_s[i] * H + j] = x_in[(size_t)(t0 + i / k) * H + j];
+        }
+    }
+}
+
+struct RouterArgs {
+    const void* x;
+    const void* w_router;
+    const void* rms_w;
+    float rms_eps;
+    void* x_norm;
+    int permute;         // 1: with a single routing block, the last CTA also permutes
+    void* xp;            //    ... and copies rows into xp when it is non-null
+    Dims d;
+    int T, tb, tt;       // routing block, tokens per CTA group
+    int do_scan, unit_width, max_units, select_only;
+    RouteBufs rb;
+    DeviceStatus st;
+};
+
+// Grid (ceil(E / 2), ceil(T / tt)), tt tokens per CTA group.  In a logits CTA
+// four warps share an expert row and take four tokens each, reading W_r, x and
+// the RMSNorm scale straight from global memory with every load of a step in
+// flight (the normalised input is never rounded before the logits).
+// The last CTA of a group (arrival counter) takes the group's Top-k (with
+// select_only the grid is (1, ceil(T / tt)) and the logits are already there).
+// Selections are counted per routing block of tb tokens (global atomics); the
+// last CTA overall scans those histograms into offsets and GEMM units.
+template <typename Tin, int VEC, int EPL>
+__global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a) {
+    extern __shared__ __align__(16) uint8_t dyn[];
+    __shared__ int hist[kMaxE];
+    __shared__ int scan_tmp[kWarps + 1];
+    __shared__ int s_flag;
+
+    const Tin* x = static_cast<const Tin*>(a.x);
+    const Tin* w_router = static_cast<const Tin*>(a.w_router);
+    const Tin* rms_w = static_cast<const Tin*>(a.rms_w);
+    RouteBufs& rb = a.rb;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int H = a.d.H, E = a.d.E, k = a.d.k;
+    const int n_groups = gridDim.x, nblocks = gridDim.y;
+    const int g = blockIdx.x, b = blockIdx.y;
+    const int t0 = b * a.tt, nt = min(a.tt, a.T - t0);
+    constexpr int kStride = 32 * VEC;
+
+    if (!a.select_only) {
+        // warp w: expert 2 g + (w >> 2), tokens 4 (w & 3) .. +3 of this group.
+        // l = sum_j W_r[e][j] x'_j with x' = x (no pre-norm) or x * g * inv_rms; the
+        // pre-norm is folded in: l = inv_rms * sum_j W_r[e][j] g_j x_j, fp32 throughout.
+        const int e = g * kEG + (warp >> 2);
+        const int tq = (warp & 3) * 4;
+        if (e < E && tq < nt) {
+            const Tin* wrow = w_router + (size_t)e * H;
+            const Tin* xr[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) xr[j] = x + (size_t)(t0 + min(tq + j, nt - 1)) * H;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f}, ss[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+            for (int c = lane * VEC; c < H; c += kStride) {
+                float wv[VEC], xv[4][VEC];
+                load_vec<Tin, VEC>(wrow + c, wv);
+                if (rms_w) {
+                    float gv[VEC];
+                    load_vec<Tin, VEC>(rms_w + c, gv);
+#pragma unroll
+                    for (int i = 0; i < VEC; ++i) wv[i] *= gv[i];
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) load_vec<Tin, VEC>(xr[j] + c, xv[j]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                    for (int i = 0; i < VEC; ++i) {
+                        acc[j] = fmaf(wv[i], xv[j][i], acc[j]);
+                        ss[j] = fmaf(xv[j][i], xv[j][i], ss[j]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+                    ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], o);
+                }
+            }
+            if (lane < 4 && tq + lane < nt) {
+                float v = acc[0], q = ss[0];
+#pragma unroll
+                for (int j = 1; j < 4; ++j) if (lane == j) { v = acc[j]; q = ss[j]; }
+                if (rms_w) v *= 1.0f / sqrtf(q / (float)H + a.rms_eps);
+                rb.logits[(size_t)(t0 + tq + lane) * E + e] = v;
+            }
+            // the first expert's warps also write the normalised tokens for the experts
+            if (rms_w && a.x_norm && e == 0) {
+                float inv[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) inv[j] = 1.0f / sqrtf(ss[j] / (float)H + a.rms_eps);
+#pragma unroll 1
+                for (int j = 0; j < 4 && tq + j < nt; ++j) {
+                    for (int c = lane * VEC; c < H; c += kStride) {
+                        float xv[VEC], gv[VEC];
+                        load_vec<Tin, VEC>(xr[j] + c, xv);
+                        load_vec<Tin, VEC>(rms_w + c, gv);
+#pragma unroll
+                        for (int i = 0; i < VEC; ++i)
+                            static_cast<Tin*>(a.x_norm)[(size_t)(t0 + tq + j) * H + c + i] =
+                                from_f32<Tin>(xv[i] * inv[j] * gv[i]);
+                    }
+                }
+            }
+        }
+        // the last logits CTA of this group continues
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) s_flag = (atomicAdd(&rb.tickets[b], 1) == n_groups - 1);
+        __syncthreads();
+        if (!s_flag) return;
+        __threadfence();
+    }
+
+    // ---- Top-k of this CTA's tokens, one warp per token; counts per routing block
+#pragma unroll 1
+    for (int tl = warp; tl < nt; tl += kWarps) {
+        const int t = t0 + tl;
+        warp_topk<EPL>(rb.logits + (size_t)t * E, E, k, t, rb,
+                       a.do_scan ? rb.block_hist + (size_t)(t / a.tb) * E : nullptr, a.st);
+    }
+    if (tid == 0 && !a.select_only) rb.tickets[b] = 0;   // every CTA of this group has arrived
+    if (!a.do_scan) return;
+
+    // ---- the last CTA scans the per-block histograms (and zeroes them for the next call)
+    __threadfence();
+    __syncthreads();
+    if (nblocks > 1) {                 // with a single CTA group this CTA is the last
+        if (tid == 0) s_flag = (atomicAdd(&rb.tickets[nblocks], 1) == nblocks - 1);
+        __syncthreads();
+        if (!s_flag) return;
+        __threadfence();
+    }
+    const int nrb = (a.T + a.tb - 1) / a.tb;              // routing blocks
+    int* chunk = reinterpret_cast<int*>(dyn);          // [kChunk][E] histogram rows
+    for (int e = tid; e < E; e += kThreads) hist[e] = 0;    // running count per expert
+#pragma unroll 1
+    for (int b0 = 0; b0 < nrb; b0 += kChunk) {
+        const int nb = min(kChunk, nrb - b0);
+        __syncthreads();
+#pragma unroll 4
+        for (int i = tid; i < nb * E; i += kThreads) {
+            chunk[i] = __ldcg(rb.block_hist + (size_t)b0 * E + i);
+            rb.block_hist[(size_t)b0 * E + i] = 0;
+        }
+        __syncthreads();
+        for (int e = tid; e < E; e += kThreads) {
+            int run = hist[e];
+#pragma unroll 1
+            for (int j = 0; j < nb; ++j) {
+                rb.block_off[(size_t)(b0 + j) * E + e] = run;
+                run += chunk[j * E + e];
+            }
+            hist[e] = run;
+        }
+    }
+    __syncthreads();
+    int* cnt = chunk;                  // counts, then offsets
+    int* ub = chunk + kMaxE;           // units per expert, then unit base
+    for (int e = tid; e < E; e += kThreads) {
+        cnt[e] = hist[e];
+        rb.counts[e] = hist[e];
+        ub[e] = (hist[e] + a.unit_width - 1) / a.unit_width;
+    }
+    __syncthreads();
+    const int total = block_exclusive_scan(cnt, E, scan_tmp);
+    int nu = block_exclusive_scan(ub, E, scan_tmp);
+    if (nu > a.max_units) {
+        if (tid == 0) report_error(a.st, kErrDeviceCheck);
+        nu = a.max_units;
+    }
+    for (int e = tid; e < E; e += kThreads) {
+        rb.offsets[e] = cnt[e];
+        const int c = hist[e];
+        for (int u = 0; u * a.unit_width < c; ++u) {
+            const int idx = ub[e] + u;
+            if (idx >= a.max_units) break;
             Unit un;
             un.expert = e;
-            un.row_start = base + u * unit_width;
-            un.n_len = min(unit_width, c - u * unit_width);
+            un.row_start = cnt[e] + u * a.unit_width;
+            un.n_len = min(a.unit_width, c - u * a.unit_width);
             un.pad = 0;
             rb.units[idx] = un;
         }
     }
+    if (tid == 0) {
+        rb.offsets[E] = total;
+        *rb.n_units = nu;
+        if (nblocks > 1) rb.tickets[nblocks] = 0;
+    }
+    if (a.permute && nrb == 1) {       // decode: permute the single routing block right here
+        __threadfence();
+        __syncthreads();
+        const Tin* x_in = a.x_norm ? static_cast<const Tin*>(a.x_norm) : x;
+        permute_block<Tin>(x_in, static_cast<Tin*>(a.xp), a.d, a.T, a.tb, 0, 0, 1, rb,
+                           reinterpret_cast<uint32_t*>(dyn + 2 * kMaxE * 4));
+    }
 }
 
-// ---------------------------------------------------------------- permute
-// One CTA per routing block of tb <= 128 tokens.  Rows of one expert are placed
-// in token order: rank = number of earlier tokens of the block that picked the
-// same expert (from a 128-bit token mask per expert) + earlier blocks' counts.
 template <typename Tin>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kThreads)
 permute_kernel(const Tin* __restrict__ x_in, Tin* __restrict__ xp, Dims d, int T, int tb,
                RouteBufs rb) {
-    extern __shared__ uint32_t bits[];   // [E][4]
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int E = d.E, k = d.k, H = d.H;
-    const int b = blockIdx.x, t0 = b * tb, nt = min(tb, T - t0);
-    for (int i = tid; i < E * 4; i += blockDim.x) bits[i] = 0;
-    __syncthreads();
-    for (int i = tid; i < nt * k; i += blockDim.x) {
-        int tl = i / k;
-        int e = rb.topk_idx[(size_t)t0 * k + i];
-        atomicOr(&bits[e * 4 + (tl >> 5)], 1u << (tl & 31));
-    }
-    __syncthreads();
-    for (int i = tid; i < nt * k; i += blockDim.x) {
-        int tl = i / k, t = t0 + tl;
-        int e = rb.topk_idx[(size_t)t0 * k + i];
-        int rank = 0;
-        for (int w = 0; w < (tl >> 5); ++w) rank += __popc(bits[e * 4 + w]);
-        rank += __popc(bits[e * 4 + (tl >> 5)] & ((1u << (tl & 31)) - 1u));
-        int pos = rb.offsets[e] + rb.block_off[(size_t)b * E + e] + rank;
-        rb.token_slot[(size_t)t0 * k + i] = pos;
-        rb.slot_token[pos] = t;
-        rb.slot_expert[pos] = e;
-    }
-    __syncthreads();
-    // copy rows: one warp per (token, slot) pair, 16-byte vectors when possible
-    const bool vec = ((H * (int)sizeof(Tin)) % 16) == 0;
-    for (int i = warp; i < nt * k; i += blockDim.x / 32) {
-        int tl = i / k;
-        int pos = rb.token_slot[(size_t)t0 * k + i];
-        const Tin* src = x_in + (size_t)(t0 + tl) * H;
-        Tin* dst = xp + (size_t)pos * H;
-        if (vec) {
-            const int nv = H * (int)sizeof(Tin) / 16;
-            const uint4* s4 = reinterpret_cast<const uint4*>(src);
-            uint4* d4 = reinterpret_cast<uint4*>(dst);
-            for (int v = lane; v < nv; v += 32) d4[v] = s4[v];
-        } else {
-            for (int j = lane; j < H; j += 32) dst[j] = src[j];
+    extern __shared__ uint32_t sm[];
+    permute_block<Tin>(x_in, xp, d, T, tb, blockIdx.x, blockIdx.y, gridDim.y, rb, sm);
+}
+
+template <typename Tin, int VEC>
+cudaError_t launch_router_t(const RouterArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
+    const int epl = (a.d.E + 31) / 32;
+    auto go = [&](auto kernel) -> cudaError_t {
+        static int allowed = 0;          // per kernel instance: dynamic smem already allowed
+        if ((int)smem > allowed) {
+            cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem);
+            if (e != cudaSuccess) return e;
+            allowed = (int)smem;
         }
-    }
+        kernel<<<grid, kThreads, smem, s>>>(a);
+        return cudaGetLastError();
+    };
+    if (epl <= 4) return go(router_kernel<Tin, VEC, 4>);
+    if (epl <= 8) return go(router_kernel<Tin, VEC, 8>);
+    return go(router_kernel<Tin, VEC, 32>);
 }
 
 }  // namespace
 
 cudaError_t launch_router(int dtype, const void* x, const void* w_router, const void* rms_w,
-                          float rms_eps, void* x_norm, const Dims& d, int T, int tb,
-                          const RouteBufs& rb, int do_scan, int unit_width, int max_units,
-                          const DeviceStatus& ds, cudaStream_t s) {
+                          float rms_eps, void* x_norm, int permute, void* xp, const Dims& d,
+                          int T, int tb, const RouteBufs& rb, int do_scan, int unit_width,
+                          int max_units, int select_only, const DeviceStatus& ds,
+                          cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
-    if (tb > kMaxTB || d.E > kMaxE || d.k > kMaxK) return cudaErrorInvalidValue;
-    dim3 grid((d.E + kEG - 1) / kEG, (T + tb - 1) / tb);
+    if (d.E > kMaxE || d.k > kMaxK || tb > 128) return cudaErrorInvalidValue;
+    const int tt = select_only ? kWarps : kMaxTB;   // select: one token per warp
+    if (!select_only && tb != kMaxTB) return cudaErrorInvalidValue;
+    RouterArgs a{x, w_router, rms_w, rms_eps, x_norm, permute, xp, d, T, tb, tt, do_scan,
+                 unit_width, max_units, select_only, rb, ds};
+    dim3 grid(select_only ? 1 : (d.E + kEG - 1) / kEG, (T + tt - 1) / tt);
+    size_t smem = (size_t)kChunk * d.E * 4;                                        // scan chunk
+    smem = std::max(smem, (size_t)2 * kMaxE * 4 + (size_t)d.E * 16 + (size_t)tb * d.k * 4);
+    if (smem > 200 * 1024) return cudaErrorInvalidValue;
     if (dtype == 0)
-        router_kernel<float><<<grid, kRouterThreads, 0, s>>>(
-            (const float*)x, (const float*)w_router, (const float*)rms_w, rms_eps,
-            (float*)x_norm, d, T, tb, rb, do_scan, unit_width, max_units, ds);
-    else
-        router_kernel<__nv_bfloat16><<<grid, kRouterThreads, 0, s>>>(
-            (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_router,
-            (const __nv_bfloat16*)rms_w, rms_eps, (__nv_bfloat16*)x_norm, d, T, tb, rb, do_scan,
-            unit_width, max_units, ds);
-    return cudaGetLastError();
+        return d.H % 4 == 0 ? launch_router_t<float, 4>(a, grid, smem, s)
+                            : launch_router_t<float, 1>(a, grid, smem, s);
+    return d.H % 8 == 0 ? launch_router_t<__nv_bfloat16, 8>(a, grid, smem, s)
+                        : launch_router_t<__nv_bfloat16, 1>(a, grid, smem, s);
 }
 
 cudaError_t launch_permute(int dtype, const void* x_in, void* xp, const Dims& d, int T, int tb,
                            const RouteBufs& rb, cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
     if (tb > 128) return cudaErrorInvalidValue;
-    int nblocks = (T + tb - 1) / tb;
-    size_t smem = (size_t)d.E * 4 * sizeof(uint32_t);
+    const int nblocks = (T + tb - 1) / tb;
+    const int split = std::max(1, std::min(16, (2 * 148 + nblocks - 1) / nblocks));   // >= 2 CTAs/SM
+    const size_t smem = (size_t)d.E * 4 * sizeof(uint32_t) + (size_t)tb * d.k * sizeof(int);
+    dim3 grid(nblocks, split);
     if (dtype == 0)
-        permute_kernel<float><<<nblocks, 256, smem, s>>>((const float*)x_in, (float*)xp, d, T, tb,
-                                                        rb);
+        permute_kernel<float><<<grid, kThreads, smem, s>>>((const float*)x_in, (float*)xp, d, T,
+                                                          tb, rb);
     else
-        permute_kernel<__nv_bfloat16><<<nblocks, 256, smem, s>>>(
+        permute_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(
             (const __nv_bfloat16*)x_in, (__nv_bfloat16*)xp, d, T, tb, rb);
     return cudaGetLastError();
 }

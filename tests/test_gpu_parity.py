@@ -64,6 +64,8 @@ SHAPES = [  # H, E, k, I, Is, T   (narrow and wide tile paths, ragged tails, k=1
     (256, 16, 4, 128, 128, 1),
     (384, 32, 8, 256, 384, 200),
     (256, 64, 6, 128, 256, 333),
+    (256, 128, 4, 128, 128, 300),     # tensor-core router (E % 128 == 0, T >= 256)
+    (128, 256, 8, 128, 0, 261),       # tensor-core router, both 128-expert panels
 ]
 
 
@@ -112,23 +114,29 @@ def test_skewed_sampled():
     assert counts[inp.skew["dead"]].sum() == 0
 
 
+STACK_MARGIN = 1e-2
+
+
 def test_stack20(record_property):
     """20 pre-RMSNorm MoE layers with residual adds, T=64.
 
-    Reference: the fp64 oracle layer by layer, with the hidden state stored in
-    bf16 between layers (the Talker's activations are bf16 tensors; each layer is
-    exact on its stored input).  Checked two ways: (1) teacher-forced, every
-    layer's oracle on the GPU's own bf16 input to that layer; (2) end to end, the
-    oracle stack from the same first input.  The drift of the GPU stack from a
-    stack that never rounds the hidden state is recorded, not asserted: bf16
-    rounding of the residual stream plus routing flips at near ties put it
-    around 3e-2 after 20 layers."""
+    (1) Teacher-forced: every layer's oracle on the GPU's own bf16 input to that
+    layer, with the single-layer contract (near-tie margin 1e-3, 2e-2 outputs).
+    (2) End to end: the oracle stack from the same first input, its hidden state
+    stored in bf16 between layers like the Talker's bf16 activations.  The two
+    stacks' inputs to layer l differ by the GPU's accumulated rounding (about
+    l * 0.3% of |h|), which moves RMS-normalised logits by up to ~6e-3; where
+    the oracle's own k-th/(k+1)-th margin is within STACK_MARGIN = 1e-2 both
+    Top-k sets are valid, so the oracle follows the GPU's set there (each such
+    set is checked to be a Top-k of the oracle logits within the margin).  The
+    final hidden state must then agree within 2e-2.  The drift from a stack that
+    never rounds its hidden state is recorded, not asserted."""
     inp = synth.make("talker_stack20")
     wl = inp.workload
     h_gpu = smt.to_device(inp.x)
     h_ref = inp.x.copy()                                          # bf16 bits
     h_f64 = synth.bf16_to_f32(inp.x).astype(np.float64)
-    worst = 0.0
+    worst, flips = 0.0, 0
     for L in inp.layers:
         layer = smt.MoELayer.from_numpy(_cfg(wl), L.arrays(), device=0)
         orc = oracle.Oracle(oracle.LayerWeights(**L.arrays(), top_k=wl.k, rms_eps=wl.rms_eps))
@@ -136,11 +144,19 @@ def test_stack20(record_property):
         y, idx, w = layer.forward(h_gpu, residual=h_gpu, return_routing=True)
         torch.cuda.synchronize()
         assert layer.check() == 0
-        rep = compare(orc, x_in, _values(y), idx.cpu().numpy(), w.cpu().numpy(), "bf16",
-                      residual=x_in)
+        idx = idx.cpu().numpy()
+        rep = compare(orc, x_in, _values(y), idx, w.cpu().numpy(), "bf16", residual=x_in)
         assert_parity(rep, "bf16")
         worst = max(worst, rep.rel_err)
-        y_ref, _, _, _ = orc.forward(h_ref, residual=h_ref)
+        logits, idx_ref, _, _ = orc.route(h_ref)
+        forced = idx_ref.copy()
+        for t in range(idx.shape[0]):
+            if set(idx[t].tolist()) != set(idx_ref[t].tolist()):
+                kth = np.sort(logits[t])[::-1][wl.k - 1]
+                assert np.all(logits[t][idx[t]] >= kth - STACK_MARGIN), (t, logits[t][idx[t]], kth)
+                forced[t] = idx[t]
+                flips += 1
+        y_ref, _, _, _ = orc.forward(h_ref, residual=h_ref, forced_idx=forced)
         h_ref = synth.bf16_bits(y_ref)
         h_f64 = h_f64 + _oracle_f64(L, wl).forward(h_f64)[0]
         h_gpu = y
@@ -151,8 +167,9 @@ def test_stack20(record_property):
     drift = np.max(np.abs(out - h_f64)) / np.max(np.abs(h_f64))
     record_property("stack_rel_err", float(err))
     record_property("worst_layer_rel_err", float(worst))
+    record_property("routing_follows", flips)
     record_property("fp64_stream_drift", float(drift))
-    assert err <= 2e-2, (err, worst, drift)
+    assert err <= 2e-2, (err, worst, flips, drift)
 
 
 def _oracle_f64(L, wl):
@@ -249,3 +266,19 @@ def test_bounded_wait_reports_timeout_and_recovers():
     layer.set_option("wait_limit_ns", 1_000_000_000)
     y, idx, w = _run(layer, inp.x)                    # the context is still usable
     assert_parity(compare(orc, inp.x, y, idx, w, "bf16"), "bf16")
+
+
+def test_route_only_tensor_core_router():
+    """moe_route at T >= 256 with E = 128 runs the tensor-core logits kernel."""
+    inp = synth.make_custom(256, 128, 6, 128, 128, 513, "bf16", seed=14)
+    layer, orc = _layer(inp)
+    idx, w = layer.route(smt.to_device(inp.x))
+    torch.cuda.synchronize()
+    _, idx_ref, w_ref, gap = orc.route(inp.x)
+    ok = gap > 1e-3
+    assert ok.sum() > 400
+    assert np.array_equal(np.sort(idx.cpu().numpy()[ok], 1), np.sort(idx_ref[ok], 1))
+    wn = w.cpu().numpy()
+    for t_ in np.nonzero(ok)[0]:
+        a = dict(zip(idx.cpu().numpy()[t_].tolist(), wn[t_].tolist()))
+        assert max(abs(a[e] - v) for e, v in zip(idx_ref[t_].tolist(), w_ref[t_].tolist())) <= 2e-5
