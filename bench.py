@@ -164,6 +164,16 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(value: float, dist=None, device=None) -> float:
+    """Largest value across ranks (the timing rule: the slowest rank sets the time)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ----------------------------------------------------------------------------- workloads
 def build_inputs(name, rank, rotate):
     """Per-copy (layers, x, residual) lists; copy 0 of rank 0 is the canonical input."""
@@ -382,11 +392,7 @@ def main():
     if world > 1:
         dist.barrier()
     ms = start.elapsed_time(end)
-    t_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = float(t.item())
+    t_max = max_over_ranks(ms, dist, dev)
     launches = int(round(launches_per_step * steps_timed))
     value = world * T * steps_timed / (t_max / 1e3)
     for hs in handles:
@@ -475,11 +481,7 @@ def main():
         e2e_step(handles[i % rotate], xh[i % rotate], yh, stream, stack, dev)
     e2.record(stream)
     torch.cuda.synchronize()
-    e_ms = s2.elapsed_time(e2)
-    if world > 1:
-        t = torch.tensor([e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
+    e_ms = max_over_ranks(s2.elapsed_time(e2), dist, dev)
     e2e = {"value": world * T * K_e2e / (e_ms / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "steps": K_e2e, "api": "moe_forward_host (pinned host buffers)"}
