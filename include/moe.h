@@ -173,6 +173,31 @@ moe_status moe_kernel_stats(moe_handle h, double* total_ms, int64_t* launches, i
 /* Free everything the handle owns (after synchronising its streams). */
 moe_status moe_destroy(moe_handle h);
 
+/*
+ * Router with no memory allocation (the pages have no counterpart: this is a
+ * deployment convenience of this library).  For callers that cannot call
+ * cudaMalloc -- e.g. a streaming audio thread that must never block, since
+ * cudaMalloc can synchronise the device and wait on driver locks, or a process
+ * whose device memory is fully reserved by another allocator -- this routes T
+ * tokens like moe_route without a handle: the caller passes the layer sizes
+ * (cfg), x [T][H] (16-byte aligned), the router weights w_router [E][H] and
+ * rms_weight [H] or NULL, all on the current device, and receives topk_idx /
+ * topk_w [T][k] (device).  The router's scratch lives in one fixed 4 MiB
+ * device array that every GPU loading this library holds until the process
+ * exits; a call needs T * E * 4 bytes of logits plus about T / 2 + 512 bytes
+ * of counters in it (T up to 8183 at E = 128); larger calls return
+ * MOE_ERR_INVALID_ARG.  Nothing is allocated or freed.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress), so make
+ * that first call before any stream capture on that device.  All calls share
+ * the array: calls whose work overlaps on the GPU (different streams, or other
+ * threads) race and must be serialised by the caller.  Logits are always
+ * formed on CUDA cores (fp32), so for T >= 256 results can differ from
+ * moe_route's tensor-core logits by rounding (near-tie tokens only).
+ */
+moe_status moe_route_noalloc(const moe_config* cfg, const void* x, const void* w_router,
+                             const void* rms_weight, int T, int32_t* topk_idx, float* topk_w,
+                             void* stream);
+
 /* Static text for a status code. */
 const char* moe_status_string(moe_status s);
 

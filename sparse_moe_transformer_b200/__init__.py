@@ -28,7 +28,7 @@ KERNEL_CLASSES = ("router", "permute", "experts", "shared", "combine")
 # Every entry point include/moe.h declares (checked by the export test).
 EXPORTS = ("moe_create", "moe_reserve", "moe_route", "moe_forward", "moe_forward_host",
            "moe_last_routing", "moe_check", "moe_set_option", "moe_kernel_stats", "moe_destroy",
-           "moe_status_string", "moe_last_error", "moe_version")
+           "moe_route_noalloc", "moe_status_string", "moe_last_error", "moe_version")
 
 
 class MoEError(RuntimeError):
@@ -67,6 +67,7 @@ def load(path: str = LIB_PATH):
         "moe_check": ([P, P], I),
         "moe_set_option": ([P, I, ctypes.c_int64], I),
         "moe_kernel_stats": ([P, P, P, I], I),
+        "moe_route_noalloc": ([ctypes.POINTER(_Config), P, P, P, I, P, P, P], I),
         "moe_destroy": ([P], I),
         "moe_status_string": ([I], ctypes.c_char_p),
         "moe_last_error": ([P], ctypes.c_char_p),

@@ -93,6 +93,11 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace
 
+namespace moe {
+// Sets the thread-local moe_last_error text (used by entry points in other files).
+void set_last_error(const char* msg) { snprintf(g_err, sizeof g_err, "%s", msg); }
+}  // namespace moe
+
 struct moe_layer {
     moe_config cfg;
     Dims d;
