@@ -140,8 +140,11 @@ typedef enum {
                                       wait targets a count that is never reached, so it
                                       runs out (test hook for the bounded-wait path)    */
     MOE_OPT_SHARED_STREAM = 2,     /* 1 (default): shared expert on the second stream   */
-    MOE_OPT_FUSE_PHASES = 3,       /* 1 (default): gate/up and down in one persistent
-                                      launch with per-tile dependency counters         */
+    MOE_OPT_FUSE_PHASES = 3,       /* 1 (default): gate/up and down in one launch: for
+                                      T*k <= 1024 a kernel whose tiles keep h on chip
+                                      and emit fp32 partial sums; otherwise one
+                                      persistent launch with per-tile dependency
+                                      counters.  0: separate launches.                */
     MOE_OPT_FORCE_SIMT = 4,        /* 1: run bf16 experts on the CUDA-core kernels      */
     MOE_OPT_KERNEL_TIMING = 5      /* 1: bracket every kernel launch with CUDA events on
                                       its own stream (read with moe_kernel_stats)       */

@@ -161,6 +161,64 @@ pack_tiles_kernel(const uint4* __restrict__ src0, const uint4* __restrict__ src1
     }
 }
 
+// One CTA per token; VEC = 8 consecutive outputs per thread.  Sum order fixed:
+// slot 0..k-1 (each the sum of its feature-block partials in block order), then
+// the shared expert, then the residual.
+__global__ void __launch_bounds__(128)
+combine_partials_kernel(const float* __restrict__ o_part, int n_blk,
+                        const __nv_bfloat16* __restrict__ sh,
+                        const __nv_bfloat16* __restrict__ res, __nv_bfloat16* __restrict__ y,
+                        const float* __restrict__ topk_w, int T, int H, int k) {
+    const int t = blockIdx.x;
+    const size_t S = (size_t)T * k;
+    for (int j0 = threadIdx.x * 8; j0 < H; j0 += blockDim.x * 8) {
+        float acc[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) acc[v] = 0.f;
+        for (int i = 0; i < k; ++i) {
+            const float w = topk_w[(size_t)t * k + i];
+            const float* src = o_part + ((size_t)t * k + i) * H + j0;
+            float4 p[2][4];                   // up to four blocks in flight
+            float sum[8];
+#pragma unroll
+            for (int v = 0; v < 8; ++v) sum[v] = 0.f;
+            for (int b0 = 0; b0 < n_blk; b0 += 4) {
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    if (b0 + b < n_blk) {
+                        const float4* q = reinterpret_cast<const float4*>(src + (b0 + b) * S * H);
+                        p[0][b] = __ldg(q);
+                        p[1][b] = __ldg(q + 1);
+                    }
+                }
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    if (b0 + b < n_blk) {
+                        sum[0] += p[0][b].x; sum[1] += p[0][b].y; sum[2] += p[0][b].z; sum[3] += p[0][b].w;
+                        sum[4] += p[1][b].x; sum[5] += p[1][b].y; sum[6] += p[1][b].z; sum[7] += p[1][b].w;
+                    }
+                }
+            }
+#pragma unroll
+            for (int v = 0; v < 8; ++v) acc[v] = fmaf(w, sum[v], acc[v]);
+        }
+        const size_t base = (size_t)t * H + j0;
+        uint4 sv = sh ? *reinterpret_cast<const uint4*>(sh + base) : make_uint4(0, 0, 0, 0);
+        uint4 rv = res ? *reinterpret_cast<const uint4*>(res + base) : make_uint4(0, 0, 0, 0);
+        const __nv_bfloat16* s8 = reinterpret_cast<const __nv_bfloat16*>(&sv);
+        const __nv_bfloat16* r8 = reinterpret_cast<const __nv_bfloat16*>(&rv);
+        __nv_bfloat16 out[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            float o = acc[v];
+            if (sh) o += __bfloat162float(s8[v]);
+            if (res) o += __bfloat162float(r8[v]);
+            out[v] = __float2bfloat16_rn(o);
+        }
+        *reinterpret_cast<uint4*>(y + base) = *reinterpret_cast<const uint4*>(out);
+    }
+}
+
 int simt_grid(size_t work) {
     size_t blocks = (work + 255) / 256;
     return (int)(blocks < 148 * 16 ? (blocks ? blocks : 1) : 148 * 16);
@@ -191,6 +249,17 @@ cudaError_t launch_combine(int dtype, const void* o, const void* sh, const void*
             combine_kernel<bf, 1><<<T, 128, 0, s>>>((const bf*)o, (const bf*)sh, (const bf*)res,
                                                     (bf*)y, topk_w, token_slot, d.H, d.k);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine_partials(const float* o_part, int n_blk, const void* shared_out,
+                                    const void* residual, void* y, const float* topk_w,
+                                    const Dims& d, int T, cudaStream_t s) {
+    if (T <= 0) return cudaSuccess;
+    if (d.H % 8) return cudaErrorInvalidValue;
+    using bf = __nv_bfloat16;
+    combine_partials_kernel<<<T, 128, 0, s>>>(o_part, n_blk, (const bf*)shared_out,
+                                              (const bf*)residual, (bf*)y, topk_w, T, d.H, d.k);
     return cudaGetLastError();
 }
 

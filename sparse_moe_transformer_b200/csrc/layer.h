@@ -144,4 +144,27 @@ cudaError_t launch_tc_experts(const TcMaps& maps, const TcArgs& a, int width, in
                               cudaStream_t s);
 int tc_smem_bytes(int width);
 
+// Few-token (decode) routed experts: one tile = one expert's tokens x one
+// 128-feature block; h stays on chip; fp32 partials o_part[I/128][T*k][H].
+struct FusedArgs {
+    const void* w_gu;          // packed gate/up tile pairs
+    const void* w_down;        // packed down tile pairs
+    const void* x_rows;        // [T][H] bf16 layer input (x or its normalised copy)
+    const int32_t* topk_idx;   // [T][k]
+    float* o_part;             // [I/128][T*k][H] fp32
+    int H, I, E, k, T;
+    int32_t* sync;             // [4]: tile counter, exit counter, an always-zero word
+    DeviceStatus st;
+    uint64_t wait_limit_ns;
+    int inject_stuck;
+};
+bool fused_supported(int H, int I, int E, int S);
+int fused_smem_bytes();
+cudaError_t launch_fused_experts(const FusedArgs& a, int grid, cudaStream_t s);
+
+// y_t = sum_j w_tj sum_b o_part[b][t k + j] + s_t [+ r_t], bf16 out.
+cudaError_t launch_combine_partials(const float* o_part, int n_blk, const void* shared_out,
+                                    const void* residual, void* y, const float* topk_w,
+                                    const Dims& d, int T, cudaStream_t s);
+
 }  // namespace moe

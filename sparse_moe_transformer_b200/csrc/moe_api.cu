@@ -119,6 +119,9 @@ struct moe_layer {
     void *hs = nullptr, *sbuf = nullptr;
     void *x_stage = nullptr, *r_stage = nullptr, *y_stage = nullptr;
     int32_t *sync_routed = nullptr, *sync_shared = nullptr, *sync_router = nullptr;
+    int32_t* sync_fused = nullptr;
+    float* o_part = nullptr;      // few-token path: [I/128][min(T*k, 1024)][H] fp32
+    bool last_fused = false;      // the last forward took the few-token path
     TcMaps routed_maps{}, shared_maps{};
     // status words
     int* err_dev = nullptr;
@@ -353,6 +356,8 @@ moe_status moe_reserve(moe_handle h, int max_tokens) {
         {(void**)&h->sync_routed, (2 + (size_t)max_units) * 4},
         {(void**)&h->sync_shared, (2 + (size_t)max_shared_units) * 4},
         {(void**)&h->sync_router, (2 + (size_t)max_shared_units) * 4},
+        {(void**)&h->sync_fused, 16},
+        {(void**)&h->o_part, h->tc_ok ? (size_t)(I / 128) * std::min<size_t>(S, 1024) * H * 4 : 0},
         {&h->x_norm, h->rms_w ? T * H * es : 0},
         {&h->xp, S * H * es},
         {&h->hbuf, S * I * es},
@@ -456,8 +461,79 @@ moe_status run_shared(moe_layer* h, const void* x_in, int T, cudaStream_t s) {
     return MOE_OK;
 }
 
+// Few-token path: route only, then one persistent kernel per feature block
+// (gate/up, SiLU*up and the down partial on chip), then the partial combine.
+moe_status run_layer_fused(moe_layer* h, const void* x, const void* residual, void* y, int T,
+                           int32_t* idx_out, float* w_out, cudaStream_t s) {
+    const Dims& d = h->d;
+    RouteBufs rb = h->rb;
+    const void* x_in = h->rms_w ? h->x_norm : x;
+    const bool side = h->shared_stream && d.Is > 0;
+    if (side && !h->rms_w) {
+        CUDA_TRY(cudaEventRecord(h->ev_fork, s));
+        CUDA_TRY(cudaStreamWaitEvent(h->s2, h->ev_fork, 0));
+        moe_status st = run_shared(h, x_in, T, h->s2);
+        if (st != MOE_OK) return st;
+        CUDA_TRY(cudaEventRecord(h->ev_join, h->s2));
+    }
+    {
+        KernelScope ks(h, MOE_KERNEL_ROUTER, s);
+        CUDA_TRY(launch_router(h->dtype, x, h->w_router, h->rms_w, h->cfg.rms_eps, h->x_norm, 0,
+                               nullptr, d, T, kRouteBlock, rb, 0, kNarrow, h->max_units, 0,
+                               h->status(), s));
+    }
+    if (side && h->rms_w) {
+        CUDA_TRY(cudaEventRecord(h->ev_fork, s));
+        CUDA_TRY(cudaStreamWaitEvent(h->s2, h->ev_fork, 0));
+        moe_status st = run_shared(h, x_in, T, h->s2);
+        if (st != MOE_OK) return st;
+        CUDA_TRY(cudaEventRecord(h->ev_join, h->s2));
+    }
+    const int S = T * d.k;
+    {
+        FusedArgs a{};
+        a.w_gu = h->w_gate; a.w_down = h->w_down; a.x_rows = x_in;
+        a.topk_idx = rb.topk_idx; a.o_part = h->o_part;
+        a.H = d.H; a.I = d.I; a.E = d.E; a.k = d.k; a.T = T;
+        a.sync = h->sync_fused; a.st = h->status(); a.wait_limit_ns = h->wait_limit_ns;
+        a.inject_stuck = h->inject_stuck;
+        const int max_units = std::min(d.E, S) + (S + 31) / 32;
+        const int grid = std::min(max_units * (d.I / 128), h->num_sms);
+        KernelScope ks(h, MOE_KERNEL_EXPERTS, s);
+        CUDA_TRY(launch_fused_experts(a, grid, s));
+        h->inject_stuck = 0;
+    }
+    if (d.Is > 0) {
+        if (side) {
+            CUDA_TRY(cudaStreamWaitEvent(s, h->ev_join, 0));
+        } else {
+            moe_status st = run_shared(h, x_in, T, s);
+            if (st != MOE_OK) return st;
+        }
+    }
+    {
+        KernelScope ks(h, MOE_KERNEL_COMBINE, s);
+        CUDA_TRY(launch_combine_partials(h->o_part, d.I / 128, d.Is > 0 ? h->sbuf : nullptr,
+                                         residual, y, rb.topk_w, d, T, s));
+    }
+    if (idx_out)
+        CUDA_TRY(cudaMemcpyAsync(idx_out, rb.topk_idx, (size_t)S * 4, cudaMemcpyDeviceToDevice, s));
+    if (w_out)
+        CUDA_TRY(cudaMemcpyAsync(w_out, rb.topk_w, (size_t)S * 4, cudaMemcpyDeviceToDevice, s));
+    h->last_T = T;
+    h->last_fused = true;
+    return MOE_OK;
+}
+
+bool use_fused(const moe_layer* h, int T) {
+    return h->tc_ok && !h->force_simt && h->fuse &&
+           fused_supported(h->d.H, h->d.I, h->d.E, T * h->d.k);
+}
+
 moe_status run_layer(moe_layer* h, const void* x, const void* residual, void* y, int T,
                      int32_t* idx_out, float* w_out, cudaStream_t s) {
+    if (use_fused(h, T)) return run_layer_fused(h, x, residual, y, T, idx_out, w_out, s);
+    h->last_fused = false;
     const Dims& d = h->d;
     const bool tc = h->tc_ok && !h->force_simt;
     const int width = choose_width(h, T);
@@ -628,6 +704,22 @@ moe_status moe_last_routing(moe_handle h, int32_t* counts, int32_t* offsets, int
     DeviceGuard g(h->device);
     cudaStream_t s = (cudaStream_t)stream;
     CUDA_TRY(cudaStreamSynchronize(s));
+    if (h->last_fused) {
+        // the few-token path builds its expert lists inside the kernel; derive the
+        // same expert-major, token-ordered bookkeeping from the recorded Top-k
+        const int E = h->d.E, k = h->d.k, S = h->last_T * k;
+        std::vector<int32_t> idx(S), cnt(E, 0), off(E + 1, 0);
+        if (S) CUDA_TRY(cudaMemcpy(idx.data(), h->rb.topk_idx, (size_t)S * 4, cudaMemcpyDeviceToHost));
+        for (int i = 0; i < S; ++i) cnt[idx[i]]++;
+        for (int e = 0; e < E; ++e) off[e + 1] = off[e] + cnt[e];
+        if (counts) memcpy(counts, cnt.data(), (size_t)E * 4);
+        if (offsets) memcpy(offsets, off.data(), (size_t)(E + 1) * 4);
+        if (token_slot) {
+            std::vector<int32_t> next(off.begin(), off.end() - 1);
+            for (int i = 0; i < S; ++i) token_slot[i] = next[idx[i]]++;
+        }
+        return MOE_OK;
+    }
     if (counts)
         CUDA_TRY(cudaMemcpy(counts, h->rb.counts, h->d.E * 4, cudaMemcpyDeviceToHost));
     if (offsets)

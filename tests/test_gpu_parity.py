@@ -49,12 +49,16 @@ def test_tiny_fp32():
     assert rep.near_ties == 0 and np.array_equal(idx, orc.forward(inp.x)[1])
 
 
-def test_decode_bf16():
+@pytest.mark.parametrize("fuse", [1, 0], ids=["few_token_kernel", "permuted_path"])
+def test_decode_bf16(fuse):
     inp = synth.make("talker_decode")
-    layer, orc = _layer(inp)
+    layer, orc = _layer(inp, fuse_phases=fuse)
     y, idx, w = _run(layer, inp.x)
     rep = compare(orc, inp.x, y, idx, w, "bf16")
     assert_parity(rep, "bf16")
+    counts, offsets, slots = layer.last_routing(inp.x.shape[0])
+    assert np.array_equal(counts, np.bincount(idx.ravel(), minlength=inp.workload.E))
+    assert np.array_equal(np.sort(slots.ravel()), np.arange(idx.size))
 
 
 SHAPES = [  # H, E, k, I, Is, T   (narrow and wide tile paths, ragged tails, k=1, no shared)
@@ -114,7 +118,10 @@ def test_skewed_sampled():
     assert counts[inp.skew["dead"]].sum() == 0
 
 
-STACK_MARGIN = 1e-2
+def _normalised(x_bits, rms_bits, eps):
+    x = synth.bf16_to_f32(x_bits).astype(np.float64)
+    g = synth.bf16_to_f32(rms_bits).astype(np.float64)
+    return x / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + eps) * g
 
 
 def test_stack20(record_property):
@@ -123,20 +130,21 @@ def test_stack20(record_property):
     (1) Teacher-forced: every layer's oracle on the GPU's own bf16 input to that
     layer, with the single-layer contract (near-tie margin 1e-3, 2e-2 outputs).
     (2) End to end: the oracle stack from the same first input, its hidden state
-    stored in bf16 between layers like the Talker's bf16 activations.  The two
-    stacks' inputs to layer l differ by the GPU's accumulated rounding (about
-    l * 0.3% of |h|), which moves RMS-normalised logits by up to ~6e-3; where
-    the oracle's own k-th/(k+1)-th margin is within STACK_MARGIN = 1e-2 both
-    Top-k sets are valid, so the oracle follows the GPU's set there (each such
-    set is checked to be a Top-k of the oracle logits within the margin).  The
-    final hidden state must then agree within 2e-2.  The drift from a stack that
+    stored in bf16 between layers like the Talker's bf16 activations.  After the
+    first layer the two stacks see slightly different inputs (bf16 rounding of
+    the residual stream), which moves a logit l_e by at most
+    b_t = max_e sum_j |W_r[e, j]| |x'_gpu[t, j] - x'_ref[t, j]| (x' the normalised
+    input); where the GPU's Top-k differs from the oracle's, each of its experts
+    must lie within 2 b_t + 1e-3 of the oracle's k-th logit (a valid Top-k of the
+    GPU's own input), and the oracle then follows the GPU's set for that token.
+    The final hidden state must agree within 2e-2.  The drift from a stack that
     never rounds its hidden state is recorded, not asserted."""
     inp = synth.make("talker_stack20")
     wl = inp.workload
     h_gpu = smt.to_device(inp.x)
     h_ref = inp.x.copy()                                          # bf16 bits
     h_f64 = synth.bf16_to_f32(inp.x).astype(np.float64)
-    worst, flips = 0.0, 0
+    worst, flips, worst_bound = 0.0, 0, 0.0
     for L in inp.layers:
         layer = smt.MoELayer.from_numpy(_cfg(wl), L.arrays(), device=0)
         orc = oracle.Oracle(oracle.LayerWeights(**L.arrays(), top_k=wl.k, rms_eps=wl.rms_eps))
@@ -149,13 +157,18 @@ def test_stack20(record_property):
         assert_parity(rep, "bf16")
         worst = max(worst, rep.rel_err)
         logits, idx_ref, _, _ = orc.route(h_ref)
+        wr = np.abs(synth.bf16_to_f32(L.w_router).astype(np.float64))
+        dx = np.abs(_normalised(x_in, L.rms_w, wl.rms_eps) - _normalised(h_ref, L.rms_w, wl.rms_eps))
+        bound = (dx @ wr.T).max(axis=1)                           # b_t for every token
         forced = idx_ref.copy()
         for t in range(idx.shape[0]):
             if set(idx[t].tolist()) != set(idx_ref[t].tolist()):
                 kth = np.sort(logits[t])[::-1][wl.k - 1]
-                assert np.all(logits[t][idx[t]] >= kth - STACK_MARGIN), (t, logits[t][idx[t]], kth)
+                margin = 2 * bound[t] + 1e-3
+                assert np.all(logits[t][idx[t]] >= kth - margin), (t, logits[t][idx[t]], kth, margin)
                 forced[t] = idx[t]
                 flips += 1
+                worst_bound = max(worst_bound, margin)
         y_ref, _, _, _ = orc.forward(h_ref, residual=h_ref, forced_idx=forced)
         h_ref = synth.bf16_bits(y_ref)
         h_f64 = h_f64 + _oracle_f64(L, wl).forward(h_f64)[0]
@@ -168,6 +181,7 @@ def test_stack20(record_property):
     record_property("stack_rel_err", float(err))
     record_property("worst_layer_rel_err", float(worst))
     record_property("routing_follows", flips)
+    record_property("largest_follow_margin", float(worst_bound))
     record_property("fp64_stream_drift", float(drift))
     assert err <= 2e-2, (err, worst, flips, drift)
 
