@@ -105,8 +105,12 @@ moe_status moe_route(moe_handle h, const void* x, int T, int32_t* topk_idx,
  * x' = x or RMSNorm(x) * g.  x, residual (nullable) and y are device [T][H] in
  * the layer dtype, 16-byte aligned.  y may alias x or residual (the inputs are
  * consumed before y is written).  topk_idx_out / topk_w_out (nullable, device
- * [T][k]) receive the routing.  The shared expert runs on a second stream of
- * the handle, joined back before the combine.  T == 0 is a no-op.
+ * [T][k]) receive the routing the call used.  T == 0 is a no-op.
+ * Few tokens (T * k <= 1024, bf16, H a multiple of 256 up to 1024, k <= 8) run
+ * as router + one expert kernel (the shared expert's blocks among its tiles) +
+ * combine, each kernel a programmatic dependent of the one before.  Larger calls
+ * run router, permutation, grouped expert GEMMs and combine, with the shared
+ * expert on a second stream of the handle, joined back before the combine.
  */
 moe_status moe_forward(moe_handle h, const void* x, const void* residual, void* y,
                        int T, int32_t* topk_idx_out, float* topk_w_out, void* stream);
@@ -139,15 +143,19 @@ typedef enum {
     MOE_OPT_INJECT_STUCK_WAIT = 1, /* 1: the next forward's first cross-tile dependency
                                       wait targets a count that is never reached, so it
                                       runs out (test hook for the bounded-wait path)    */
-    MOE_OPT_SHARED_STREAM = 2,     /* 1 (default): shared expert on the second stream   */
+    MOE_OPT_SHARED_STREAM = 2,     /* 1 (default): shared expert on the second stream
+                                      (the few-token kernel runs it among its tiles)    */
     MOE_OPT_FUSE_PHASES = 3,       /* 1 (default): gate/up and down in one launch: for
                                       T*k <= 1024 a kernel whose tiles keep h on chip
-                                      and emit fp32 partial sums; otherwise one
+                                      and emit fp32 partial sums (the shared expert's
+                                      blocks among them); otherwise one
                                       persistent launch with per-tile dependency
                                       counters.  0: separate launches.                */
     MOE_OPT_FORCE_SIMT = 4,        /* 1: run bf16 experts on the CUDA-core kernels      */
     MOE_OPT_KERNEL_TIMING = 5      /* 1: bracket every kernel launch with CUDA events on
-                                      its own stream (read with moe_kernel_stats)       */
+                                      its own stream (read with moe_kernel_stats); this
+                                      also turns off the programmatic launch overlap of
+                                      the few-token path, so each kernel is timed alone */
 } moe_option;
 
 /* Set an option; takes effect at the next call.  Errors: INVALID_ARG. */

@@ -161,62 +161,68 @@ pack_tiles_kernel(const uint4* __restrict__ src0, const uint4* __restrict__ src1
     }
 }
 
-// One CTA per token; VEC = 8 consecutive outputs per thread.  Sum order fixed:
-// slot 0..k-1 (each the sum of its feature-block partials in block order), then
-// the shared expert, then the residual.
-__global__ void __launch_bounds__(128)
-combine_partials_kernel(const float* __restrict__ o_part, int n_blk,
-                        const __nv_bfloat16* __restrict__ sh,
-                        const __nv_bfloat16* __restrict__ res, __nv_bfloat16* __restrict__ y,
+// y_t = sum_j w_tj (sum_b o_part[b][t k + j]) + sum_b o_part[b][T k + t] [+ r_t].
+// Eight threads (lanes 8 g .. 8 g + 7 of a warp) share 4 columns of one token
+// (k <= 8): thread s takes routed slot j = s (the sum of its block partials in
+// block order, times w_tj) and the shared expert's blocks b = s, s + 8, ...; the
+// eight values are then added in a fixed butterfly order, so the result does not
+// depend on timing.  Every load of a thread is issued before its first add.
+constexpr int kCombineSub = 8;
+constexpr int kCombineMaxLoads = 16;
+__global__ void __launch_bounds__(256)
+combine_partials_kernel(const float* __restrict__ o_part, int n_blk, int n_blk_s,
+                        const __nv_bfloat16* res, __nv_bfloat16* y,
                         const float* __restrict__ topk_w, int T, int H, int k) {
-    const int t = blockIdx.x;
-    const size_t S = (size_t)T * k;
-    for (int j0 = threadIdx.x * 8; j0 < H; j0 += blockDim.x * 8) {
-        float acc[8];
+    grid_dependency_wait();                    // partials of the expert kernel
+    grid_dependents_launch();                  // the next router may start its prologue
+    const int per_t = H / 4;
+    const int gid = blockIdx.x * (blockDim.x / kCombineSub) + threadIdx.x / kCombineSub;
+    const int sub = threadIdx.x % kCombineSub;
+    const bool live = gid < T * per_t;
+    const int t = live ? gid / per_t : 0, c4 = live ? (gid - t * per_t) * 4 : 0;
+    const size_t S = (size_t)T * k, bstride = (S + T) * H;
+    // thread `sub` holds routed slot j = sub (k <= kCombineSub: at most one) as
+    // items 0 .. n_r - 1, then shared blocks sub, sub + 8, ... as the next items
+    const bool has_slot = live && sub < k;
+    const int n_r = has_slot ? n_blk : 0;
+    const int n_s = live && sub < n_blk_s ? (n_blk_s - sub + kCombineSub - 1) / kCombineSub : 0;
+    const float* pr = o_part + ((size_t)t * k + sub) * H + c4;
+    const float* ps = o_part + (S + t) * H + c4 + (size_t)sub * bstride;
+    const float w = has_slot ? __ldg(topk_w + (size_t)t * k + sub) : 0.f;
+    float4 v[kCombineMaxLoads];
 #pragma unroll
-        for (int v = 0; v < 8; ++v) acc[v] = 0.f;
-        for (int i = 0; i < k; ++i) {
-            const float w = topk_w[(size_t)t * k + i];
-            const float* src = o_part + ((size_t)t * k + i) * H + j0;
-            float4 p[2][4];                   // up to four blocks in flight
-            float sum[8];
-#pragma unroll
-            for (int v = 0; v < 8; ++v) sum[v] = 0.f;
-            for (int b0 = 0; b0 < n_blk; b0 += 4) {
-#pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    if (b0 + b < n_blk) {
-                        const float4* q = reinterpret_cast<const float4*>(src + (b0 + b) * S * H);
-                        p[0][b] = __ldg(q);
-                        p[1][b] = __ldg(q + 1);
-                    }
-                }
-#pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    if (b0 + b < n_blk) {
-                        sum[0] += p[0][b].x; sum[1] += p[0][b].y; sum[2] += p[0][b].z; sum[3] += p[0][b].w;
-                        sum[4] += p[1][b].x; sum[5] += p[1][b].y; sum[6] += p[1][b].z; sum[7] += p[1][b].w;
-                    }
-                }
-            }
-#pragma unroll
-            for (int v = 0; v < 8; ++v) acc[v] = fmaf(w, sum[v], acc[v]);
-        }
-        const size_t base = (size_t)t * H + j0;
-        uint4 sv = sh ? *reinterpret_cast<const uint4*>(sh + base) : make_uint4(0, 0, 0, 0);
-        uint4 rv = res ? *reinterpret_cast<const uint4*>(res + base) : make_uint4(0, 0, 0, 0);
-        const __nv_bfloat16* s8 = reinterpret_cast<const __nv_bfloat16*>(&sv);
-        const __nv_bfloat16* r8 = reinterpret_cast<const __nv_bfloat16*>(&rv);
-        __nv_bfloat16 out[8];
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-            float o = acc[v];
-            if (sh) o += __bfloat162float(s8[v]);
-            if (res) o += __bfloat162float(r8[v]);
-            out[v] = __float2bfloat16_rn(o);
-        }
-        *reinterpret_cast<uint4*>(y + base) = *reinterpret_cast<const uint4*>(out);
+    for (int i = 0; i < kCombineMaxLoads; ++i) {
+        if (i < n_r) v[i] = __ldg(reinterpret_cast<const float4*>(pr + (size_t)i * bstride));
+        else if (i < n_r + n_s)
+            v[i] = __ldg(reinterpret_cast<const float4*>(ps + (size_t)(i - n_r) * kCombineSub * bstride));
     }
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f), sh = sum;
+#pragma unroll
+    for (int i = 0; i < kCombineMaxLoads; ++i) {
+        if (i < n_r) { sum.x += v[i].x; sum.y += v[i].y; sum.z += v[i].z; sum.w += v[i].w; }
+        else if (i < n_r + n_s) { sh.x += v[i].x; sh.y += v[i].y; sh.z += v[i].z; sh.w += v[i].w; }
+    }
+    float4 acc = make_float4(fmaf(w, sum.x, sh.x), fmaf(w, sum.y, sh.y), fmaf(w, sum.z, sh.z),
+                             fmaf(w, sum.w, sh.w));
+#pragma unroll
+    for (int o = 1; o < kCombineSub; o <<= 1) {
+        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
+        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+    }
+    if (!live || sub != 0) return;
+    float o[4] = {acc.x, acc.y, acc.z, acc.w};
+    __nv_bfloat16 out[4];
+    if (res) {
+        const uint2 rv = *reinterpret_cast<const uint2*>(res + (size_t)t * H + c4);
+        const __nv_bfloat16* r4 = reinterpret_cast<const __nv_bfloat16*>(&rv);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) o[q] += __bfloat162float(r4[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) out[q] = __float2bfloat16_rn(o[q]);
+    *reinterpret_cast<uint2*>(y + (size_t)t * H + c4) = *reinterpret_cast<const uint2*>(out);
 }
 
 int simt_grid(size_t work) {
@@ -252,15 +258,28 @@ cudaError_t launch_combine(int dtype, const void* o, const void* sh, const void*
     return cudaGetLastError();
 }
 
-cudaError_t launch_combine_partials(const float* o_part, int n_blk, const void* shared_out,
+cudaError_t launch_combine_partials(const float* o_part, int n_blk, int n_blk_s,
                                     const void* residual, void* y, const float* topk_w,
-                                    const Dims& d, int T, cudaStream_t s) {
+                                    const Dims& d, int T, int pdl, cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
-    if (d.H % 8) return cudaErrorInvalidValue;
+    if (d.H % 4 || n_blk < 1) return cudaErrorInvalidValue;
+    // loads per thread: its slot's blocks plus its shared blocks
+    if (d.k > kCombineSub || n_blk + (n_blk_s + kCombineSub - 1) / kCombineSub > kCombineMaxLoads)
+        return cudaErrorInvalidValue;
     using bf = __nv_bfloat16;
-    combine_partials_kernel<<<T, 128, 0, s>>>(o_part, n_blk, (const bf*)shared_out,
-                                              (const bf*)residual, (bf*)y, topk_w, T, d.H, d.k);
-    return cudaGetLastError();
+    const int groups = T * (d.H / 4);
+    const int per_block = 256 / kCombineSub;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((groups + per_block - 1) / per_block);
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, combine_partials_kernel, o_part, n_blk, n_blk_s,
+                              (const bf*)residual, (bf*)y, topk_w, T, d.H, d.k);
 }
 
 cudaError_t launch_simt_gate_up(int dtype, const void* xin, const void* w_gate, const void* w_up,

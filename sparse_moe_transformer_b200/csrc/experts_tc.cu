@@ -457,6 +457,9 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
     }
 
     // ------------------------------------------------ teardown
+    // The MMA role runs on lane 0 of warp 1 only: reconverge every warp before
+    // the CTA barrier (bar.sync expects whole warps).
+    __syncwarp();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();

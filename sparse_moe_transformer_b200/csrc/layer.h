@@ -54,11 +54,13 @@ struct RouteBufs {
 // select_only the logits already sit in rb.logits (tensor-core router).
 // With permute and a single routing block (T <= tb) the last CTA also performs
 // the permutation (what launch_permute would do; the row copy only if xp != null).
+// pdl: launch as a programmatic dependent of the previous kernel in the stream
+// (the router waits on the device for it before reading anything).
 cudaError_t launch_router(int dtype, const void* x, const void* w_router, const void* rms_w,
                           float rms_eps, void* x_norm, int permute, void* xp, const Dims& d,
                           int T, int tb, const RouteBufs& rb, int do_scan, int unit_width,
                           int max_units, int select_only, const DeviceStatus& st,
-                          cudaStream_t s);
+                          cudaStream_t s, int pdl = 0);
 
 // Expert-contiguous order of the token rows: fills token_slot / slot_token /
 // slot_expert, and gathers the rows into xp unless xp is null.
@@ -104,6 +106,7 @@ __host__ __device__ inline size_t packed_down_elems(int E, int H, int I) {
 cudaError_t launch_pack_tiles(const void* src0, const void* src1, void* dst, int E, int R, int C,
                               cudaStream_t s);
 
+
 // CUDA-core expert kernels (exact fp32 accumulate; any shape).
 // rows: permuted rows (routed) or tokens (shared, slot_expert == nullptr).
 // packed: weights are in the tile-contiguous layout (gate/up in one buffer).
@@ -144,27 +147,34 @@ cudaError_t launch_tc_experts(const TcMaps& maps, const TcArgs& a, int width, in
                               cudaStream_t s);
 int tc_smem_bytes(int width);
 
-// Few-token (decode) routed experts: one tile = one expert's tokens x one
-// 128-feature block; h stays on chip; fp32 partials o_part[I/128][T*k][H].
+// Few-token (decode) experts: one tile = the tokens of one expert (or of the
+// shared expert) x one 128-feature block; h stays on chip; fp32 partials
+// o_part[b][row][H] with rows 0..T*k-1 the routed slots t*k+j and rows
+// T*k+t the shared expert's tokens.
 struct FusedArgs {
-    const void* w_gu;          // packed gate/up tile pairs
-    const void* w_down;        // packed down tile pairs
+    const void* w_gu;          // routed packed gate/up tile pairs
+    const void* w_down;        // routed packed down tile pairs
+    const void* ws_gu;         // shared-expert packed gate/up (Is > 0)
+    const void* ws_down;       // shared-expert packed down (Is > 0)
     const void* x_rows;        // [T][H] bf16 layer input (x or its normalised copy)
-    const int32_t* topk_idx;   // [T][k]
-    float* o_part;             // [I/128][T*k][H] fp32
-    int H, I, E, k, T;
-    int32_t* sync;             // [4]: tile counter, exit counter, an always-zero word
+    const int32_t* topk_idx;   // [T][k] from the router
+    float* o_part;             // [max(I, Is) / 128][T*k + T][H] fp32
+    int H, I, Is, E, k, T;
+    int x_early;               // 1: x_rows exists before the router runs (no pre-norm)
+    const int32_t* zero_word;  // a word that stays 0 (bounded-wait test hook)
     DeviceStatus st;
     uint64_t wait_limit_ns;
     int inject_stuck;
 };
-bool fused_supported(int H, int I, int E, int S);
+bool fused_supported(int H, int I, int Is, int E, int k, int S);
 int fused_smem_bytes();
-cudaError_t launch_fused_experts(const FusedArgs& a, int grid, cudaStream_t s);
+int fused_unit_rows();     // token rows per tile
+// pdl: launch as a programmatic dependent of the previous kernel in the stream.
+cudaError_t launch_fused_experts(const FusedArgs& a, int grid, int pdl, cudaStream_t s);
 
-// y_t = sum_j w_tj sum_b o_part[b][t k + j] + s_t [+ r_t], bf16 out.
-cudaError_t launch_combine_partials(const float* o_part, int n_blk, const void* shared_out,
+// y_t = sum_j w_tj sum_b o_part[b][t k + j] + sum_b o_part[b][T k + t] [+ r_t], bf16 out.
+cudaError_t launch_combine_partials(const float* o_part, int n_blk, int n_blk_s,
                                     const void* residual, void* y, const float* topk_w,
-                                    const Dims& d, int T, cudaStream_t s);
+                                    const Dims& d, int T, int pdl, cudaStream_t s);
 
 }  // namespace moe

@@ -120,7 +120,7 @@ struct moe_layer {
     void *x_stage = nullptr, *r_stage = nullptr, *y_stage = nullptr;
     int32_t *sync_routed = nullptr, *sync_shared = nullptr, *sync_router = nullptr;
     int32_t* sync_fused = nullptr;
-    float* o_part = nullptr;      // few-token path: [I/128][min(T*k, 1024)][H] fp32
+    float* o_part = nullptr;      // few-token path: [max(I, Is)/128][T*k + T][H] fp32
     bool last_fused = false;      // the last forward took the few-token path
     TcMaps routed_maps{}, shared_maps{};
     // status words
@@ -357,7 +357,9 @@ moe_status moe_reserve(moe_handle h, int max_tokens) {
         {(void**)&h->sync_shared, (2 + (size_t)max_shared_units) * 4},
         {(void**)&h->sync_router, (2 + (size_t)max_shared_units) * 4},
         {(void**)&h->sync_fused, 16},
-        {(void**)&h->o_part, h->tc_ok ? (size_t)(I / 128) * std::min<size_t>(S, 1024) * H * 4 : 0},
+        {(void**)&h->o_part, h->tc_ok ? (size_t)(std::max(I, Is) / 128) *
+                                            (std::min<size_t>(S, 1024) + std::min<size_t>(T, 1024)) * H * 4
+                                      : 0},
         {&h->x_norm, h->rms_w ? T * H * es : 0},
         {&h->xp, S * H * es},
         {&h->hbuf, S * I * es},
@@ -461,60 +463,47 @@ moe_status run_shared(moe_layer* h, const void* x_in, int T, cudaStream_t s) {
     return MOE_OK;
 }
 
-// Few-token path: route only, then one persistent kernel per feature block
-// (gate/up, SiLU*up and the down partial on chip), then the partial combine.
+// Few-token path: route only, then one persistent kernel over the feature
+// blocks of the shared expert and of the selected experts (gate/up, SiLU*up and
+// the down partial on chip), then the partial combine.  The expert kernel and
+// the combine are programmatic dependents: each starts while its predecessor
+// finishes and waits on the device for the predecessor's results.
 moe_status run_layer_fused(moe_layer* h, const void* x, const void* residual, void* y, int T,
                            int32_t* idx_out, float* w_out, cudaStream_t s) {
     const Dims& d = h->d;
     RouteBufs rb = h->rb;
     const void* x_in = h->rms_w ? h->x_norm : x;
-    const bool side = h->shared_stream && d.Is > 0;
-    if (side && !h->rms_w) {
-        CUDA_TRY(cudaEventRecord(h->ev_fork, s));
-        CUDA_TRY(cudaStreamWaitEvent(h->s2, h->ev_fork, 0));
-        moe_status st = run_shared(h, x_in, T, h->s2);
-        if (st != MOE_OK) return st;
-        CUDA_TRY(cudaEventRecord(h->ev_join, h->s2));
-    }
+    // with per-kernel timing on, events separate the kernels and the overlap is off
+    const int pdl = h->timing ? 0 : 1;
     {
         KernelScope ks(h, MOE_KERNEL_ROUTER, s);
         CUDA_TRY(launch_router(h->dtype, x, h->w_router, h->rms_w, h->cfg.rms_eps, h->x_norm, 0,
                                nullptr, d, T, kRouteBlock, rb, 0, kNarrow, h->max_units, 0,
-                               h->status(), s));
-    }
-    if (side && h->rms_w) {
-        CUDA_TRY(cudaEventRecord(h->ev_fork, s));
-        CUDA_TRY(cudaStreamWaitEvent(h->s2, h->ev_fork, 0));
-        moe_status st = run_shared(h, x_in, T, h->s2);
-        if (st != MOE_OK) return st;
-        CUDA_TRY(cudaEventRecord(h->ev_join, h->s2));
+                               h->status(), s, pdl));
     }
     const int S = T * d.k;
     {
         FusedArgs a{};
-        a.w_gu = h->w_gate; a.w_down = h->w_down; a.x_rows = x_in;
+        a.w_gu = h->w_gate; a.w_down = h->w_down;
+        a.ws_gu = d.Is ? h->ws_gate : nullptr; a.ws_down = d.Is ? h->ws_down : nullptr;
+        a.x_rows = x_in; a.x_early = h->rms_w ? 0 : 1;
         a.topk_idx = rb.topk_idx; a.o_part = h->o_part;
-        a.H = d.H; a.I = d.I; a.E = d.E; a.k = d.k; a.T = T;
-        a.sync = h->sync_fused; a.st = h->status(); a.wait_limit_ns = h->wait_limit_ns;
+        a.H = d.H; a.I = d.I; a.Is = d.Is; a.E = d.E; a.k = d.k; a.T = T;
+        a.zero_word = h->sync_fused + 2;
+        a.st = h->status(); a.wait_limit_ns = h->wait_limit_ns;
         a.inject_stuck = h->inject_stuck;
-        const int max_units = std::min(d.E, S) + (S + 31) / 32;
-        const int grid = std::min(max_units * (d.I / 128), h->num_sms);
+        const int unit_rows = fused_unit_rows();
+        const int max_units = std::min(d.E, S) + (S + unit_rows - 1) / unit_rows;
+        const int tiles = max_units * (d.I / 128) + (T + unit_rows - 1) / unit_rows * (d.Is / 128);
+        const int grid = std::min(tiles, h->num_sms);
         KernelScope ks(h, MOE_KERNEL_EXPERTS, s);
-        CUDA_TRY(launch_fused_experts(a, grid, s));
+        CUDA_TRY(launch_fused_experts(a, grid, pdl, s));
         h->inject_stuck = 0;
-    }
-    if (d.Is > 0) {
-        if (side) {
-            CUDA_TRY(cudaStreamWaitEvent(s, h->ev_join, 0));
-        } else {
-            moe_status st = run_shared(h, x_in, T, s);
-            if (st != MOE_OK) return st;
-        }
     }
     {
         KernelScope ks(h, MOE_KERNEL_COMBINE, s);
-        CUDA_TRY(launch_combine_partials(h->o_part, d.I / 128, d.Is > 0 ? h->sbuf : nullptr,
-                                         residual, y, rb.topk_w, d, T, s));
+        CUDA_TRY(launch_combine_partials(h->o_part, d.I / 128, d.Is / 128, residual, y, rb.topk_w,
+                                         d, T, pdl, s));
     }
     if (idx_out)
         CUDA_TRY(cudaMemcpyAsync(idx_out, rb.topk_idx, (size_t)S * 4, cudaMemcpyDeviceToDevice, s));
@@ -527,7 +516,7 @@ moe_status run_layer_fused(moe_layer* h, const void* x, const void* residual, vo
 
 bool use_fused(const moe_layer* h, int T) {
     return h->tc_ok && !h->force_simt && h->fuse &&
-           fused_supported(h->d.H, h->d.I, h->d.E, T * h->d.k);
+           fused_supported(h->d.H, h->d.I, h->d.Is, h->d.E, h->d.k, T * h->d.k);
 }
 
 moe_status run_layer(moe_layer* h, const void* x, const void* residual, void* y, int T,

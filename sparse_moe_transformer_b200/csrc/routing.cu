@@ -20,6 +20,7 @@
 
 #include "device.cuh"
 #include "layer.h"
+#include "topk.cuh"
 
 namespace moe {
 namespace {
@@ -75,18 +76,22 @@ __device__ int block_exclusive_scan(int* v, int n, int* tmp) {
     return total;
 }
 
-// Order-preserving map of an fp32 value to uint32 (larger float -> larger key;
-// -0 and +0 map to the same key, so they tie like equal values).
-__device__ __forceinline__ uint32_t order_key(float f) {
-    const uint32_t u = __float_as_uint(f + 0.0f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+// Top-k of one token (one warp), written to the routing buffers; the
+// selections are counted into the token's routing block (hist = its row, nullable).
+template <int EPL>
+__device__ void warp_topk_vals(const float (&lv)[EPL], int E, int k, int t, RouteBufs& rb,
+                               int* hist, const DeviceStatus& st) {
+    const int lane = threadIdx.x & 31;
+    int my_e;
+    float my_w;
+    warp_topk_select<EPL>(lv, E, k, my_e, my_w, st);
+    if (lane < k) {
+        rb.topk_idx[(size_t)t * k + lane] = my_e;
+        rb.topk_w[(size_t)t * k + lane] = my_w;
+        if (hist) atomicAdd(hist + my_e, 1);
+    }
 }
 
-// Top-k of one token (one warp): EPL logits per lane (experts lane + 32 i).
-// Each round: every lane proposes its best unselected expert; the warp takes
-// the largest key (redux.sync max) and, among equal keys, the lowest expert
-// index (redux.sync min) -- the lower-index tie rule.  The selections are
-// counted into the token's routing block (hist = its row, nullable).
 template <int EPL>
 __device__ void warp_topk(const float* lrow, int E, int k, int t, RouteBufs& rb, int* hist,
                           const DeviceStatus& st) {
@@ -95,41 +100,7 @@ __device__ void warp_topk(const float* lrow, int E, int k, int t, RouteBufs& rb,
 #pragma unroll
     for (int i = 0; i < EPL; ++i)
         lv[i] = (lane + 32 * i < E) ? __ldcg(lrow + lane + 32 * i) : -INFINITY;
-    uint32_t taken = 0;                 // bit i: element lane + 32 i already selected
-    float vmax = 0.f, z = 0.f, my_v = 0.f;
-    int my_e = -1;
-#pragma unroll 1
-    for (int r = 0; r < k; ++r) {
-        uint32_t bk = 0;
-        int bi = 0x7fffffff;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            const int e = lane + 32 * i;
-            const uint32_t key = order_key(lv[i]);
-            if (e < E && !(taken & (1u << i)) && (bi == 0x7fffffff || key > bk)) { bk = key; bi = e; }
-        }
-        const uint32_t kmax = __reduce_max_sync(0xffffffffu, bk);
-        int e_win = (int)__reduce_min_sync(0xffffffffu, (bi != 0x7fffffff && bk == kmax)
-                                                            ? (uint32_t)bi : 0xffffffffu);
-        if (e_win < 0 || e_win >= E) {            // cannot happen for k <= E
-            if (lane == 0) report_error(st, kErrDeviceCheck);
-            e_win = r;
-        }
-        if ((e_win & 31) == lane) taken |= 1u << (e_win >> 5);
-        float bv = 0.f;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) if (lane + 32 * i == e_win) bv = lv[i];
-        bv = __shfl_sync(0xffffffffu, bv, e_win & 31);
-        if (r == 0) vmax = bv;
-        const float ex = expf(bv - vmax);
-        z += ex;
-        if (lane == r) { my_e = e_win; my_v = ex; }   // lane r keeps selection r
-    }
-    if (lane < k) {
-        rb.topk_idx[(size_t)t * k + lane] = my_e;
-        rb.topk_w[(size_t)t * k + lane] = my_v / z;
-        if (hist) atomicAdd(hist + my_e, 1);
-    }
+    warp_topk_vals<EPL>(lv, E, k, t, rb, hist, st);
 }
 
 // Permutation of routing block b (tb <= 128 tokens): rows of one expert in token
@@ -229,6 +200,11 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a) {
     __shared__ int scan_tmp[kWarps + 1];
     __shared__ int s_flag;
 
+    // Launched as a programmatic dependent, wait for the producer of x before
+    // touching anything; then let the next kernel (the few-token expert kernel,
+    // which waits on the device for this grid's results) start its prologue.
+    grid_dependency_wait();
+    grid_dependents_launch();
     const Tin* x = static_cast<const Tin*>(a.x);
     const Tin* w_router = static_cast<const Tin*>(a.w_router);
     const Tin* rms_w = static_cast<const Tin*>(a.rms_w);
@@ -410,7 +386,7 @@ permute_kernel(const Tin* __restrict__ x_in, Tin* __restrict__ xp, Dims d, int T
 }
 
 template <typename Tin, int VEC>
-cudaError_t launch_router_t(const RouterArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
+cudaError_t launch_router_t(const RouterArgs& a, dim3 grid, size_t smem, int pdl, cudaStream_t s) {
     const int epl = (a.d.E + 31) / 32;
     auto go = [&](auto kernel) -> cudaError_t {
         static int allowed = 0;          // per kernel instance: dynamic smem already allowed
@@ -420,8 +396,17 @@ cudaError_t launch_router_t(const RouterArgs& a, dim3 grid, size_t smem, cudaStr
             if (e != cudaSuccess) return e;
             allowed = (int)smem;
         }
-        kernel<<<grid, kThreads, smem, s>>>(a);
-        return cudaGetLastError();
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = pdl ? 1 : 0;
+        return cudaLaunchKernelEx(&cfg, kernel, a);
     };
     if (epl <= 4) return go(router_kernel<Tin, VEC, 4>);
     if (epl <= 8) return go(router_kernel<Tin, VEC, 8>);
@@ -434,7 +419,7 @@ cudaError_t launch_router(int dtype, const void* x, const void* w_router, const 
                           float rms_eps, void* x_norm, int permute, void* xp, const Dims& d,
                           int T, int tb, const RouteBufs& rb, int do_scan, int unit_width,
                           int max_units, int select_only, const DeviceStatus& ds,
-                          cudaStream_t s) {
+                          cudaStream_t s, int pdl) {
     if (T <= 0) return cudaSuccess;
     if (d.E > kMaxE || d.k > kMaxK || tb > 128) return cudaErrorInvalidValue;
     const int tt = select_only ? kWarps : kMaxTB;   // select: one token per warp
@@ -446,10 +431,10 @@ cudaError_t launch_router(int dtype, const void* x, const void* w_router, const 
     smem = std::max(smem, (size_t)2 * kMaxE * 4 + (size_t)d.E * 16 + (size_t)tb * d.k * 4);
     if (smem > 200 * 1024) return cudaErrorInvalidValue;
     if (dtype == 0)
-        return d.H % 4 == 0 ? launch_router_t<float, 4>(a, grid, smem, s)
-                            : launch_router_t<float, 1>(a, grid, smem, s);
-    return d.H % 8 == 0 ? launch_router_t<__nv_bfloat16, 8>(a, grid, smem, s)
-                        : launch_router_t<__nv_bfloat16, 1>(a, grid, smem, s);
+        return d.H % 4 == 0 ? launch_router_t<float, 4>(a, grid, smem, pdl, s)
+                            : launch_router_t<float, 1>(a, grid, smem, pdl, s);
+    return d.H % 8 == 0 ? launch_router_t<__nv_bfloat16, 8>(a, grid, smem, pdl, s)
+                        : launch_router_t<__nv_bfloat16, 1>(a, grid, smem, pdl, s);
 }
 
 cudaError_t launch_permute(int dtype, const void* x_in, void* xp, const Dims& d, int T, int tb,

@@ -70,6 +70,9 @@ SHAPES = [  # H, E, k, I, Is, T   (narrow and wide tile paths, ragged tails, k=1
     (256, 64, 6, 128, 256, 333),
     (256, 128, 4, 128, 128, 300),     # tensor-core router (E % 128 == 0, T >= 256)
     (128, 256, 8, 128, 0, 261),       # tensor-core router, both 128-expert panels
+    (256, 128, 6, 128, 128, 16),      # few-token kernel: shared expert one full token tile
+    (512, 256, 8, 256, 0, 9),         # ... 256 experts, k = 8, no shared expert
+    (256, 128, 4, 128, 256, 17),      # ... shared expert over two token tiles
 ]
 
 
