@@ -92,17 +92,19 @@ def source_sha(path):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def recorded_traffic(workload):
-    """DRAM bytes per launch of the routed-expert kernel from a committed ncu summary,
-    valid only while the kernel source is unchanged since the capture."""
+def recorded_traffic(workload, kernel):
+    """DRAM bytes per launch of the roofline kernel from a committed ncu summary,
+    valid only while that kernel's source file is unchanged since the capture."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    src = os.path.join(ROOT, "sparse_moe_transformer_b200", "csrc", "experts_tc.cu")
     e = d.get(workload)
-    if not e or e.get("experts_tc_sha") != source_sha(src):
+    if not e or e.get("kernel") != kernel:
+        return None
+    src = os.path.join(ROOT, "sparse_moe_transformer_b200", "csrc", e["source"])
+    if not os.path.exists(src) or e.get("source_sha") != source_sha(src):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -427,12 +429,22 @@ def main():
     kern = {c: {"launches": n, "mean_us": (t / n * 1e3) if n else None}
             for c, (n, t) in per_class.items()}
 
-    # ---- roofline of the dominant kernel (routed experts)
+    # ---- roofline of the dominant kernel (the expert kernel)
     peaks = load_peaks()
     ex_n, ex_ms = per_class.get("experts", (0, 0.0))
     ex_s = (ex_ms / ex_n) / 1e3 if ex_n else None
     e_bytes = float(np.mean([w["experts_bytes"] for w in work]))
     e_flops = float(np.mean([w["experts_flops"] for w in work]))
+    # no permutation and no shared-expert launch: the few-token kernel ran, and its
+    # tiles include the shared expert's blocks (weights once, all T tokens)
+    few_token = per_class.get("permute", (0, 0))[0] == 0 and per_class.get("shared", (0, 0))[0] == 0
+    if few_token:
+        es = 2 if wl.dtype == "bf16" else 4
+        e_bytes += 3 * wl.H * wl.Is * es
+        e_flops += 2 * 3 * wl.H * wl.Is * T
+        kname = "tc_fused_experts_kernel"
+    else:
+        kname = "tc_routed_experts_kernel"
     t_mem = e_bytes / (peaks["hbm_gbs"] * 1e9)
     t_tc = e_flops / (peaks["bf16_tflops"] * 1e12)
     if ex_s:
@@ -444,8 +456,9 @@ def main():
             achieved = e_flops / ex_s / 1e12
             roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
-        roof["traffic"] = recorded_traffic(name)
-        roof["kernel"] = "tc_experts_kernel (routed experts, gate/up + down in one launch)"
+        roof["traffic"] = recorded_traffic(name, kname)
+        roof["kernel"] = kname + (" (few-token tiles: routed + shared experts, h on chip)"
+                                  if few_token else " (grouped routed experts, gate/up + down)")
         roof["algorithmic_per_launch"] = e_bytes if roof["bound"] == "hbm" else e_flops
         roof["mean_launch_us"] = ex_s * 1e6
         roof["peak_source"] = peaks["source"] + (" burst" if roof["bound"] == "tensor" else "")
