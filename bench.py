@@ -435,16 +435,14 @@ def main():
     ex_s = (ex_ms / ex_n) / 1e3 if ex_n else None
     e_bytes = float(np.mean([w["experts_bytes"] for w in work]))
     e_flops = float(np.mean([w["experts_flops"] for w in work]))
-    # no permutation and no shared-expert launch: the few-token kernel ran, and its
-    # tiles include the shared expert's blocks (weights once, all T tokens)
-    few_token = per_class.get("permute", (0, 0))[0] == 0 and per_class.get("shared", (0, 0))[0] == 0
-    if few_token:
+    # no shared-expert launch: the expert kernel's tiles include the shared expert
+    # (its weights once, every token); no permutation either: the few-token kernel
+    few_token = per_class.get("permute", (0, 0))[0] == 0
+    if wl.Is and per_class.get("shared", (0, 0))[0] == 0:
         es = 2 if wl.dtype == "bf16" else 4
-        e_bytes += 3 * wl.H * wl.Is * es
+        e_bytes += 3 * wl.H * wl.Is * es + (0 if few_token else 2 * T * wl.H * es)
         e_flops += 2 * 3 * wl.H * wl.Is * T
-        kname = "tc_fused_experts_kernel"
-    else:
-        kname = "tc_routed_experts_kernel"
+    kname = "tc_fused_experts_kernel" if few_token else "tc_routed_experts_kernel"
     t_mem = e_bytes / (peaks["hbm_gbs"] * 1e9)
     t_tc = e_flops / (peaks["bf16_tflops"] * 1e12)
     if ex_s:
@@ -458,7 +456,7 @@ def main():
                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
         roof["traffic"] = recorded_traffic(name, kname)
         roof["kernel"] = kname + (" (few-token tiles: routed + shared experts, h on chip)"
-                                  if few_token else " (grouped routed experts, gate/up + down)")
+                                  if few_token else " (grouped routed + shared expert tiles)")
         roof["algorithmic_per_launch"] = e_bytes if roof["bound"] == "hbm" else e_flops
         roof["mean_launch_us"] = ex_s * 1e6
         roof["peak_source"] = peaks["source"] + (" burst" if roof["bound"] == "tensor" else "")

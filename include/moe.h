@@ -109,8 +109,8 @@ moe_status moe_route(moe_handle h, const void* x, int T, int32_t* topk_idx,
  * Few tokens (T * k <= 1024, bf16, H a multiple of 256 up to 1024, k <= 8) run
  * as router + one expert kernel (the shared expert's blocks among its tiles) +
  * combine, each kernel a programmatic dependent of the one before.  Larger calls
- * run router, permutation, grouped expert GEMMs and combine, with the shared
- * expert on a second stream of the handle, joined back before the combine.
+ * run router, permutation, one grouped expert GEMM launch (the shared expert's
+ * tiles among the routed experts') and combine.
  */
 moe_status moe_forward(moe_handle h, const void* x, const void* residual, void* y,
                        int T, int32_t* topk_idx_out, float* topk_w_out, void* stream);
@@ -143,8 +143,9 @@ typedef enum {
     MOE_OPT_INJECT_STUCK_WAIT = 1, /* 1: the next forward's first cross-tile dependency
                                       wait targets a count that is never reached, so it
                                       runs out (test hook for the bounded-wait path)    */
-    MOE_OPT_SHARED_STREAM = 2,     /* 1 (default): shared expert on the second stream
-                                      (the few-token kernel runs it among its tiles)    */
+    MOE_OPT_SHARED_STREAM = 2,     /* 1 (default): on the CUDA-core path the shared
+                                      expert runs on the second stream (the tensor-core
+                                      kernels run it among their own tiles)            */
     MOE_OPT_FUSE_PHASES = 3,       /* 1 (default): gate/up and down in one launch: for
                                       T*k <= 1024 a kernel whose tiles keep h on chip
                                       and emit fp32 partial sums (the shared expert's

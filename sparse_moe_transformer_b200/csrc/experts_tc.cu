@@ -19,7 +19,9 @@
 // warps read TMEM with tcgen05.ld and store bf16 rows with 16-byte stores.
 //
 // The kernel is persistent: CTAs take tiles from a global counter, gate/up tiles
-// first, then down tiles.  When both phases run in one launch, a down tile of a
+// first, then down tiles.  A launch may carry a second, dense problem -- the
+// shared expert over every token -- whose tiles interleave as [routed gate/up |
+// shared gate/up | routed down | shared down].  When both phases run in one launch, a down tile of a
 // unit waits (bounded by a time limit) until the unit's gate/up tiles have
 // published their h rows; every gate/up tile is taken before any down tile and
 // never waits, so the wait always ends.  (Ordering tiles in waves of units --
@@ -69,7 +71,8 @@ struct TcCfg {
 };
 
 struct Tile {
-    int phase;       // 0 gate/up, 1 down, -1 no more work
+    int phase;       // 0 gate/up, 1 down, 2 router logits, -1 no more work
+    int prob;        // 0: the launch's first problem, 1: the second (dense) problem
     int unit;
     int mt;          // 128-row block of the weight matrix
     int expert;
@@ -77,11 +80,16 @@ struct Tile {
     int n_len;       // activation rows (MMA N before rounding to 16)
 };
 
-__device__ __forceinline__ Tile decode_tile(int i, int n_units, const TcArgs& a, int mt_gu,
-                                            int mt_dn, int bn) {
+// Tile list: [problem 0 gate/up | problem 1 gate/up | problem 0 down | problem 1 down]
+// (router launches: one two-panel tile of 256 experts per unit).  Every gate/up
+// tile comes before every down tile, so a down tile's wait for its unit's h always
+// ends.  n0 / n1: units of the two problems; mt_gu0 / mt_gu1 their gate/up blocks.
+__device__ __forceinline__ Tile decode_tile(int i, int n0, int n1, const TcArgs& a, int mt_gu0,
+                                            int mt_gu1, int mt_dn, int bn) {
     Tile t;
-    if (a.phases == 4) {          // router logits: one two-panel tile (256 experts) per unit
-        if (i < n_units * mt_dn) {
+    t.prob = 0;
+    if (a.phases == 4) {
+        if (i < n0 * mt_dn) {
             t.phase = 2; t.unit = i / mt_dn; t.mt = i - t.unit * mt_dn;
             t.expert = 0; t.row_start = t.unit * bn; t.n_len = min(bn, a.dense_T - t.row_start);
         } else {
@@ -89,28 +97,38 @@ __device__ __forceinline__ Tile decode_tile(int i, int n_units, const TcArgs& a,
         }
         return t;
     }
-    {
-        const int n_gu = (a.phases & 1) ? n_units * mt_gu : 0;
-        const int n_dn = (a.phases & 2) ? n_units * mt_dn : 0;
-        if (i < n_gu) {
-            t.phase = 0; t.unit = i / mt_gu; t.mt = i - t.unit * mt_gu;
-        } else if (i - n_gu < n_dn) {
-            const int j = i - n_gu;
-            t.phase = 1; t.unit = j / mt_dn; t.mt = j - t.unit * mt_dn;
-        } else {
-            t.phase = -1; t.unit = t.mt = t.expert = t.row_start = t.n_len = 0;
-            return t;
-        }
+    const int g0 = (a.phases & 1) ? n0 * mt_gu0 : 0, g1 = (a.phases & 1) ? n1 * mt_gu1 : 0;
+    const int d0 = (a.phases & 2) ? n0 * mt_dn : 0, d1 = (a.phases & 2) ? n1 * mt_dn : 0;
+    if (i < g0) {
+        t.phase = 0; t.unit = i / mt_gu0; t.mt = i - t.unit * mt_gu0;
+    } else if ((i -= g0) < g1) {
+        t.phase = 0; t.prob = 1; t.unit = i / mt_gu1; t.mt = i - t.unit * mt_gu1;
+    } else if ((i -= g1) < d0) {
+        t.phase = 1; t.unit = i / mt_dn; t.mt = i - t.unit * mt_dn;
+    } else if ((i -= d0) < d1) {
+        t.phase = 1; t.prob = 1; t.unit = i / mt_dn; t.mt = i - t.unit * mt_dn;
+    } else {
+        t.phase = -1; t.unit = t.mt = t.expert = t.row_start = t.n_len = 0;
+        return t;
     }
-    if (a.dense_T > 0) {
+    const int dense = t.prob ? a.dense2_T : a.dense_T;
+    if (dense > 0) {
         t.expert = 0;
         t.row_start = t.unit * bn;
-        t.n_len = min(bn, a.dense_T - t.row_start);
+        t.n_len = min(bn, dense - t.row_start);
     } else {
         const Unit u = a.units[t.unit];
         t.expert = u.expert; t.row_start = u.row_start; t.n_len = u.n_len;
     }
     return t;
+}
+
+// Down and router tiles cover two 128-row blocks; with an odd number of blocks the
+// last tile's second block is the packed layout's zero fill and is neither loaded
+// nor multiplied.
+__device__ __forceinline__ bool single_panel(const Tile& t, const TcArgs& a) {
+    const int rows = t.phase == 1 ? a.H : t.phase == 2 ? a.I : 0;
+    return rows && (2 * t.mt + 1) * kBM >= rows;
 }
 
 // Wait (bounded) until `flag` reaches `target`; false after recording a timeout.
@@ -149,19 +167,22 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool router = a.phases == 4;
-    const int mt_gu = a.I / kBM;                      // gate/up tiles: 128 features each
+    const int mt_gu0 = a.I / kBM;                     // gate/up tiles: 128 features each
+    const int mt_gu1 = a.dense2_T > 0 ? a.I2 / kBM : 1;
     // down tiles: 256 output features each; router tiles: 256 experts each
     const int mt_dn = router ? (a.I / kBM + 1) / 2 : (a.H / kBM + 1) / 2;
-    const int kb_gu = a.H / kBK, kb_dn = router ? a.H / kBK : a.I / kBK;
+    const int kb_gu = a.H / kBK;
+    const int kb_dn0 = router ? a.H / kBK : a.I / kBK, kb_dn1 = a.I2 / kBK;
     int* tile_counter = a.sync;
     int* exit_counter = a.sync + 1;
-    int* done = a.sync + 2;
     const uint64_t limit = a.wait_limit_ns;
     const bool fused = (a.phases & 3) == 3;
 
     const int n_units = a.dense_T > 0 ? (a.dense_T + BN - 1) / BN : *a.n_units;
+    const int n_units2 = a.dense2_T > 0 ? (a.dense2_T + BN - 1) / BN : 0;
     const int n_tiles = router ? n_units * mt_dn
-                               : n_units * (((a.phases & 1) ? mt_gu : 0) + ((a.phases & 2) ? mt_dn : 0));
+                               : ((a.phases & 1) ? n_units * mt_gu0 + n_units2 * mt_gu1 : 0) +
+                                 ((a.phases & 2) ? (n_units + n_units2) * mt_dn : 0);
 
     if (tid == 0) {
         for (int s = 0; s < C::kStages; ++s) { mbar_init(&full[s], 2); mbar_init(&empty[s], 1); }
@@ -175,6 +196,7 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
         mbar_fence_init();
         tma_prefetch_desc(&maps.b_x);
         tma_prefetch_desc(&maps.b_h);
+        if (a.dense2_T > 0) { tma_prefetch_desc(&maps.b_x2); tma_prefetch_desc(&maps.b_h2); }
     }
     if (warp == 1) tmem_alloc(tmem_slot, C::kTmemCols);
     tc_fence_before();
@@ -202,7 +224,7 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
             int i = n_tiles;
             if (lane == 0 && ok && !error_pending(a.st)) i = atomicAdd(tile_counter, 1);
             i = __shfl_sync(0xffffffffu, i, 0);
-            Tile t = decode_tile(i, n_units, a, mt_gu, mt_dn, BN);
+            Tile t = decode_tile(i, n_units, n_units2, a, mt_gu0, mt_gu1, mt_dn, BN);
             const int r = tc % kRing;
             int w_ok = 1;
             if (lane == 0) {
@@ -212,16 +234,26 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
             if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
             ++tc;
             if (t.phase < 0) break;
-            const bool gather = BN <= 32 && t.phase == 0 && a.row_token != nullptr;
+            const bool p1 = t.prob == 1;
+            const bool gather = BN <= 32 && t.phase == 0 && !p1 && a.row_token != nullptr;
             const int nb16 = (t.n_len + kBoxRows - 1) / kBoxRows;
+            const int mt_gu = p1 ? mt_gu1 : mt_gu0;
+            const int kb_dn = p1 ? kb_dn1 : kb_dn0;
             const int KB = t.phase == 0 ? kb_gu : kb_dn;
-            const uint32_t a_bytes = 2 * kABytes;     // a tile pair per k-step
+            // a tile pair per k-step; the zero-filled second panel of an odd count of
+            // 128-row blocks (W_down with odd H / 128, W_r with odd E / 128) is skipped
+            const uint32_t a_stride = 2 * kABytes;
+            const uint32_t a_bytes = single_panel(t, a) ? kABytes : a_stride;
             const uint32_t bytes = a_bytes + (gather ? 0 : nb16 * kBoxBytes);
+            const uint8_t* wg = p1 ? static_cast<const uint8_t*>(a.w_gu2) : w_gu;
+            const uint8_t* wd = p1 ? static_cast<const uint8_t*>(a.w_down2) : w_dn;
             const uint8_t* a_src =
-                t.phase == 0 ? w_gu + (size_t)(t.expert * mt_gu + t.mt) * kb_gu * a_bytes
-                : t.phase == 1 ? w_dn + (size_t)(t.expert * mt_dn + t.mt) * kb_dn * a_bytes
-                               : w_gu + (size_t)t.mt * kb_dn * a_bytes;   // packed W_r
-            const CUtensorMap* bmap = t.phase == 1 ? &maps.b_h : &maps.b_x;
+                t.phase == 0 ? wg + (size_t)(t.expert * mt_gu + t.mt) * kb_gu * a_stride
+                : t.phase == 1 ? wd + (size_t)(t.expert * mt_dn + t.mt) * kb_dn * a_stride
+                               : w_gu + (size_t)t.mt * kb_dn * a_stride;   // packed W_r
+            const CUtensorMap* bmap = t.phase == 1 ? (p1 ? &maps.b_h2 : &maps.b_h)
+                                                   : (p1 ? &maps.b_x2 : &maps.b_x);
+            int* done = p1 ? a.done2 : a.sync + 2;
             // gather mode: lane covers (row, 16-byte chunk) pairs p = lane + 32 j
             const __nv_bfloat16* src_row[8];
             uint4 nx[8];
@@ -247,7 +279,7 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
                     if (!mbar_wait(&empty[s], ((q / C::kStages) & 1) ^ 1, a.st, limit)) fail = 1;
                     else {
                         mbar_arrive_expect_tx(&full[s], bytes);
-                        bulk_load(smem + s * C::kStageBytes, a_src + (size_t)kb * a_bytes, a_bytes,
+                        bulk_load(smem + s * C::kStageBytes, a_src + (size_t)kb * a_stride, a_bytes,
                                   &full[s], pol_w);
                     }
                 }
@@ -280,7 +312,7 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
                     if (!mbar_wait(&empty[s], ((it / C::kStages) & 1) ^ 1, a.st, limit)) fail = 1;
                     else {
                         mbar_arrive_expect_tx(&full[s], bytes);
-                        bulk_load(A0, a_src + (size_t)kb * a_bytes, a_bytes, &full[s], pol_w);
+                        bulk_load(A0, a_src + (size_t)kb * a_stride, a_bytes, &full[s], pol_w);
                         if (!gather)
                             for (int j = 0; j < nb16; ++j)
                                 tma_load_2d(B + j * kBoxBytes, bmap, &full[s], kb * kBK,
@@ -331,7 +363,8 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
             const uint32_t idesc = idesc_bf16_f32(kBM, N);
             const uint32_t d_gate = tmem_base + acc * 2 * BN;
             const uint32_t d_up = d_gate + BN;
-            const int KB = t.phase == 0 ? kb_gu : kb_dn;
+            const int KB = t.phase == 0 ? kb_gu : (t.prob ? kb_dn1 : kb_dn0);
+            const bool one = single_panel(t, a);
             bool fail = false;
             for (int kb = 0; kb < KB; ++kb, ++it) {
                 const int s = it % C::kStages;
@@ -346,7 +379,7 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
                     const uint32_t accum = (kb | kk) != 0;
                     // gate/up: (gate, up) panels; down: two 128-row output blocks
                     tc_mma_bf16(d_gate, smem_desc_sw128(a0 + kk * 32), bd, idesc, accum);
-                    tc_mma_bf16(d_up, smem_desc_sw128(a1 + kk * 32), bd, idesc, accum);
+                    if (!one) tc_mma_bf16(d_up, smem_desc_sw128(a1 + kk * 32), bd, idesc, accum);
                 }
                 tc_commit(&empty[s]);   // frees the stage once these MMAs have read it
             }
@@ -365,8 +398,7 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
         const int q = warp & 3;
         const int half = ew >> 2;
         __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(epi_smem + ew * kEpiStage);
-        __nv_bfloat16* hbuf = static_cast<__nv_bfloat16*>(a.hbuf);
-        __nv_bfloat16* outb = static_cast<__nv_bfloat16*>(a.out);
+
         int tc = 0, ac = 0, pub = 0;
         while (true) {
             const int r = tc % kRing;
@@ -388,8 +420,9 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
                 // router logits: logits[rows][256 mt + 128 p + 32 q + lane], fp32
                 const int e0 = t.mt * 2 * kBM + q * 32 + lane;
                 float* lg = a.logits + (size_t)t.row_start * a.I;
+                const int rpanels = single_panel(t, a) ? 1 : 2;
                 for (int c = half; c < nc; c += 2) {
-                    for (int p = 0; p < 2; ++p) {
+                    for (int p = 0; p < rpanels; ++p) {
                         float v[16];
                         tmem_ld16((p ? tu : tg) + c * 16, v);
                         tmem_wait_ld();
@@ -405,11 +438,12 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
                 ++ac;
                 continue;
             }
-            const int ld = t.phase == 0 ? a.I : a.H;
+            const int ld = t.phase == 0 ? (t.prob ? a.I2 : a.I) : a.H;
             const int col0 = t.phase == 0 ? t.mt * kBM : t.mt * 2 * kBM;
             const int panels = t.phase == 0 ? 1 : (col0 + kBM < a.H ? 2 : 1);
-            __nv_bfloat16* dst = (t.phase == 0 ? hbuf : outb) + (size_t)t.row_start * ld + col0 +
-                                 q * 32;
+            void* base = t.phase == 0 ? (t.prob ? a.hbuf2 : a.hbuf) : (t.prob ? a.out2 : a.out);
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(base) + (size_t)t.row_start * ld +
+                                 col0 + q * 32;
             for (int c = half; c < nc; c += 2) {
                 for (int p = 0; p < panels; ++p) {
                     float v[16];
@@ -449,6 +483,7 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
                 __syncwarp();
                 if (lane == 0) mbar_arrive(pubbar);
                 if (ew == 0 && lane == 0) {
+                    int* done = t.prob ? a.done2 : a.sync + 2;
                     if (mbar_wait(pubbar, pub & 1, a.st, limit)) red_release_gpu_add(done + t.unit, 1);
                 }
                 ++pub;
@@ -472,7 +507,8 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
     __syncthreads();
     if (s_misc[0]) {   // last CTA out: reset the counters for the next launch
         __threadfence();
-        for (int u = tid; u < n_units; u += kThreads) done[u] = 0;
+        for (int u = tid; u < n_units; u += kThreads) a.sync[2 + u] = 0;
+        for (int u = tid; u < n_units2; u += kThreads) a.done2[u] = 0;
         if (tid == 0) { *tile_counter = 0; *exit_counter = 0; }
     }
 }
@@ -534,6 +570,8 @@ cudaError_t launch_tc_experts(const TcMaps& maps, const TcArgs& a, int width, in
                               cudaStream_t s) {
     if (grid <= 0) return cudaSuccess;
     if (a.H % kBM || a.I % kBM) return cudaErrorInvalidValue;   // I, H multiples of 128
+    if (a.dense2_T > 0 && (a.I2 % kBM || !a.w_gu2 || !a.w_down2 || !a.done2))
+        return cudaErrorInvalidValue;
     if (width == 32) return launch_width<32>(maps, a, grid, s);
     if (width == 256) return launch_width<256>(maps, a, grid, s);
     return cudaErrorInvalidValue;

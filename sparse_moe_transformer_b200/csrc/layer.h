@@ -119,7 +119,8 @@ cudaError_t launch_simt_down(int dtype, const void* hbuf, const void* w_down, in
 
 // tcgen05 grouped SwiGLU expert GEMM (bf16, fp32 accumulate).
 struct TcMaps {
-    CUtensorMap b_x, b_h; // activations [rows][H], [rows][I], 16-row boxes, 128-byte swizzle
+    CUtensorMap b_x, b_h;   // activations [rows][H], [rows][I], 16-row boxes, 128-byte swizzle
+    CUtensorMap b_x2, b_h2; // the second (dense) problem's, when TcArgs::dense2_T > 0
 };
 struct TcArgs {
     const void* w_gu;     // packed gate/up tiles (see packed_gu_offset); router: packed W_r
@@ -141,6 +142,16 @@ struct TcArgs {
     DeviceStatus st;
     uint64_t wait_limit_ns;
     int inject_stuck;
+    // A second, dense problem in the same launch (the shared expert: every row of
+    // x, weights w_gu2 / w_down2 packed like an expert's, intermediate size I2).
+    // Its gate/up tiles follow the first problem's, its down tiles follow the first
+    // problem's down tiles.  dense2_T == 0: none.
+    const void* w_gu2;
+    const void* w_down2;
+    int I2, dense2_T;
+    void* hbuf2;         // [dense2_T][I2] bf16
+    void* out2;          // [dense2_T][H] bf16
+    int32_t* done2;      // [ceil(dense2_T / width)] per-unit counters (self-resetting)
 };
 // width: 32 (decode) or 256 (prefill) tile-width instance.
 cudaError_t launch_tc_experts(const TcMaps& maps, const TcArgs& a, int width, int grid,

@@ -530,7 +530,11 @@ moe_status run_layer(moe_layer* h, const void* x, const void* residual, void* y,
     if (idx_out) rb.topk_idx = idx_out;
     if (w_out) rb.topk_w = w_out;
     const void* x_in = h->rms_w ? h->x_norm : x;
-    const bool side = h->shared_stream && d.Is > 0;
+    // tensor cores: the shared expert's tiles join the routed experts' launch (two
+    // persistent kernels would only compete for the SMs; on a side stream it held
+    // every SM while the router waited).  CUDA cores: optionally a second stream.
+    const bool merged = tc && d.Is > 0;
+    const bool side = !merged && h->shared_stream && d.Is > 0;
 
     if (side && !h->rms_w) {     // the shared expert needs only x: start it right away
         CUDA_TRY(cudaEventRecord(h->ev_fork, s));
@@ -578,16 +582,27 @@ moe_status run_layer(moe_layer* h, const void* x, const void* residual, void* y,
         a.st = h->status(); a.wait_limit_ns = h->wait_limit_ns;
         a.inject_stuck = h->inject_stuck && h->fuse;
         const int max_units = std::min(h->max_units, (S + width - 1) / width + d.E);
-        const int tiles = max_units * (d.I / 128 + (d.H / 128 + 1) / 2);
+        int tiles = max_units * (d.I / 128 + (d.H / 128 + 1) / 2);
+        TcMaps maps = h->routed_maps;
+        if (merged) {
+            a.w_gu2 = h->ws_gate; a.w_down2 = h->ws_down;
+            a.I2 = d.Is; a.dense2_T = T;
+            a.hbuf2 = h->hs; a.out2 = h->sbuf;
+            a.done2 = h->sync_shared + 2;
+            maps.b_h2 = h->shared_maps.b_h;
+            moe_status st = make_map(&maps.b_x2, x_in, (uint64_t)T, d.H, 16);
+            if (st != MOE_OK) return st;
+            tiles += (T + width - 1) / width * (d.Is / 128 + (d.H / 128 + 1) / 2);
+        }
         const int grid = std::min(tiles, h->num_sms);
         {
             KernelScope ks(h, MOE_KERNEL_EXPERTS, s);
-            CUDA_TRY(launch_tc_experts(h->routed_maps, a, width, grid, s));
+            CUDA_TRY(launch_tc_experts(maps, a, width, grid, s));
         }
         if (!h->fuse) {
             a.phases = 2;
             KernelScope ks(h, MOE_KERNEL_EXPERTS, s);
-            CUDA_TRY(launch_tc_experts(h->routed_maps, a, width, grid, s));
+            CUDA_TRY(launch_tc_experts(maps, a, width, grid, s));
         }
         h->inject_stuck = 0;
     } else {
@@ -601,7 +616,7 @@ moe_status run_layer(moe_layer* h, const void* x, const void* residual, void* y,
         CUDA_TRY(launch_simt_down(h->dtype, h->hbuf, h->w_down, h->tc_ok, rb.slot_expert, n_rows,
                                   S, d.H, d.I, h->obuf, s));
     }
-    if (d.Is > 0) {
+    if (d.Is > 0 && !merged) {
         if (side) {
             CUDA_TRY(cudaStreamWaitEvent(s, h->ev_join, 0));
         } else {

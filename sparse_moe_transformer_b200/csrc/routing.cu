@@ -201,8 +201,20 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a) {
     __shared__ int s_flag;
 
     // Launched as a programmatic dependent, wait for the producer of x before
-    // touching anything; then let the next kernel (the few-token expert kernel,
-    // which waits on the device for this grid's results) start its prologue.
+    // touching anything it writes; then let the next kernel (the few-token expert
+    // kernel, which waits on the device for this grid's results) start its
+    // prologue.  The router rows are constants: their L2 prefetch goes first.
+    if (!a.select_only && threadIdx.x == 0 && blockIdx.y == 0) {
+        const int e0 = blockIdx.x * kEG;
+        const int ne = min(kEG, a.d.E - e0);
+        const size_t row_bytes = (size_t)a.d.H * sizeof(Tin);
+        const Tin* wr = static_cast<const Tin*>(a.w_router) + (size_t)e0 * a.d.H;
+        auto aligned16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+        if (ne > 0 && (row_bytes * ne) % 16 == 0 && aligned16(wr))
+            prefetch_l2_bulk(wr, (uint32_t)(row_bytes * ne));
+        if (a.rms_w && row_bytes % 16 == 0 && blockIdx.x == 0 && aligned16(a.rms_w))
+            prefetch_l2_bulk(a.rms_w, (uint32_t)row_bytes);
+    }
     grid_dependency_wait();
     grid_dependents_launch();
     const Tin* x = static_cast<const Tin*>(a.x);
