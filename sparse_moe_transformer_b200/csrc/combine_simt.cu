@@ -23,9 +23,11 @@ namespace {
 
 template <typename T, int VEC>
 __global__ void __launch_bounds__(128)
-combine_kernel(const T* __restrict__ o, const T* __restrict__ sh, const T* __restrict__ res,
-               T* __restrict__ y, const float* __restrict__ topk_w,
+combine_kernel(const T* __restrict__ o, const T* __restrict__ sh, const T* res, T* y,
+               const float* __restrict__ topk_w,
                const int32_t* __restrict__ token_slot, int H, int k) {
+    grid_dependency_wait();          // expert outputs of the previous kernel
+    grid_dependents_launch();
     const int t = blockIdx.x;
     __shared__ int slot[16];
     __shared__ float wt[16];
@@ -234,28 +236,33 @@ int simt_grid(size_t work) {
 
 cudaError_t launch_combine(int dtype, const void* o, const void* sh, const void* res, void* y,
                            const float* topk_w, const int32_t* token_slot, const Dims& d, int T,
-                           cudaStream_t s) {
+                           cudaStream_t s, int pdl) {
     if (T <= 0) return cudaSuccess;
     if (d.k > 16) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(T);
+    cfg.blockDim = dim3(128);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    using bf = __nv_bfloat16;
     if (dtype == 0) {
+        const float *o_ = (const float*)o, *sh_ = (const float*)sh, *res_ = (const float*)res;
         if (d.H % 4 == 0)
-            combine_kernel<float, 4><<<T, 128, 0, s>>>((const float*)o, (const float*)sh,
-                                                       (const float*)res, (float*)y, topk_w,
-                                                       token_slot, d.H, d.k);
-        else
-            combine_kernel<float, 1><<<T, 128, 0, s>>>((const float*)o, (const float*)sh,
-                                                       (const float*)res, (float*)y, topk_w,
-                                                       token_slot, d.H, d.k);
-    } else {
-        using bf = __nv_bfloat16;
-        if (d.H % 8 == 0)
-            combine_kernel<bf, 8><<<T, 128, 0, s>>>((const bf*)o, (const bf*)sh, (const bf*)res,
-                                                    (bf*)y, topk_w, token_slot, d.H, d.k);
-        else
-            combine_kernel<bf, 1><<<T, 128, 0, s>>>((const bf*)o, (const bf*)sh, (const bf*)res,
-                                                    (bf*)y, topk_w, token_slot, d.H, d.k);
+            return cudaLaunchKernelEx(&cfg, combine_kernel<float, 4>, o_, sh_, res_, (float*)y,
+                                      topk_w, token_slot, d.H, d.k);
+        return cudaLaunchKernelEx(&cfg, combine_kernel<float, 1>, o_, sh_, res_, (float*)y, topk_w,
+                                  token_slot, d.H, d.k);
     }
-    return cudaGetLastError();
+    const bf *o_ = (const bf*)o, *sh_ = (const bf*)sh, *res_ = (const bf*)res;
+    if (d.H % 8 == 0)
+        return cudaLaunchKernelEx(&cfg, combine_kernel<bf, 8>, o_, sh_, res_, (bf*)y, topk_w,
+                                  token_slot, d.H, d.k);
+    return cudaLaunchKernelEx(&cfg, combine_kernel<bf, 1>, o_, sh_, res_, (bf*)y, topk_w,
+                              token_slot, d.H, d.k);
 }
 
 cudaError_t launch_combine_partials(const float* o_part, int n_blk, int n_blk_s,

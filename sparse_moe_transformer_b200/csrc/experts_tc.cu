@@ -203,6 +203,10 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // launched as a programmatic dependent: the set-up above overlapped the previous
+    // kernel; from here on its results (units, activations) are read
+    grid_dependency_wait();
+    grid_dependents_launch();
 
     if (warp == 0) {
         // ------------------------------------------------ scheduler + copy producer
@@ -534,7 +538,7 @@ tc_router_logits_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
 }
 
 template <int BN>
-cudaError_t launch_width(const TcMaps& maps, const TcArgs& a, int grid, cudaStream_t s) {
+cudaError_t launch_width(const TcMaps& maps, const TcArgs& a, int grid, int pdl, cudaStream_t s) {
     static bool configured = false;   // per process; the attribute is per function
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(tc_routed_experts_kernel<BN>,
@@ -551,13 +555,19 @@ cudaError_t launch_width(const TcMaps& maps, const TcArgs& a, int grid, cudaStre
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    if (a.phases == 4)
-        tc_router_logits_kernel<BN><<<grid, kThreads, TcCfg<BN>::kSmem, s>>>(maps, a);
-    else if (a.dense_T > 0)
-        tc_shared_expert_kernel<BN><<<grid, kThreads, TcCfg<BN>::kSmem, s>>>(maps, a);
-    else
-        tc_routed_experts_kernel<BN><<<grid, kThreads, TcCfg<BN>::kSmem, s>>>(maps, a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = TcCfg<BN>::kSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (a.phases == 4) return cudaLaunchKernelEx(&cfg, tc_router_logits_kernel<BN>, maps, a);
+    if (a.dense_T > 0) return cudaLaunchKernelEx(&cfg, tc_shared_expert_kernel<BN>, maps, a);
+    return cudaLaunchKernelEx(&cfg, tc_routed_experts_kernel<BN>, maps, a);
 }
 
 }  // namespace
@@ -567,13 +577,13 @@ int tc_smem_bytes(int width) {
 }
 
 cudaError_t launch_tc_experts(const TcMaps& maps, const TcArgs& a, int width, int grid,
-                              cudaStream_t s) {
+                              cudaStream_t s, int pdl) {
     if (grid <= 0) return cudaSuccess;
     if (a.H % kBM || a.I % kBM) return cudaErrorInvalidValue;   // I, H multiples of 128
     if (a.dense2_T > 0 && (a.I2 % kBM || !a.w_gu2 || !a.w_down2 || !a.done2))
         return cudaErrorInvalidValue;
-    if (width == 32) return launch_width<32>(maps, a, grid, s);
-    if (width == 256) return launch_width<256>(maps, a, grid, s);
+    if (width == 32) return launch_width<32>(maps, a, grid, pdl, s);
+    if (width == 256) return launch_width<256>(maps, a, grid, pdl, s);
     return cudaErrorInvalidValue;
 }
 

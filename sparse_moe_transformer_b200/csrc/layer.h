@@ -65,12 +65,12 @@ cudaError_t launch_router(int dtype, const void* x, const void* w_router, const 
 // Expert-contiguous order of the token rows: fills token_slot / slot_token /
 // slot_expert, and gathers the rows into xp unless xp is null.
 cudaError_t launch_permute(int dtype, const void* x_in, void* xp, const Dims& d, int T, int tb,
-                           const RouteBufs& rb, cudaStream_t s);
+                           const RouteBufs& rb, cudaStream_t s, int pdl = 0);
 
 // y = [residual +] s + sum_j w_tj * o[token_slot[t][j]]
 cudaError_t launch_combine(int dtype, const void* o, const void* shared_out, const void* residual,
                            void* y, const float* topk_w, const int32_t* token_slot,
-                           const Dims& d, int T, cudaStream_t s);
+                           const Dims& d, int T, cudaStream_t s, int pdl = 0);
 
 // Tile-contiguous weight layout of the tensor-core path.  A weight matrix
 // [E][R][C] is cut into 128-row x 64-column tiles, each stored as the exact
@@ -154,8 +154,9 @@ struct TcArgs {
     int32_t* done2;      // [ceil(dense2_T / width)] per-unit counters (self-resetting)
 };
 // width: 32 (decode) or 256 (prefill) tile-width instance.
+// pdl: launch as a programmatic dependent of the previous kernel in the stream.
 cudaError_t launch_tc_experts(const TcMaps& maps, const TcArgs& a, int width, int grid,
-                              cudaStream_t s);
+                              cudaStream_t s, int pdl = 0);
 int tc_smem_bytes(int width);
 
 // Few-token (decode) experts: one tile = the tokens of one expert (or of the

@@ -407,7 +407,7 @@ bool use_tc_router(const moe_layer* h, int T) {
 }
 
 moe_status run_tc_router(moe_layer* h, const void* x, int T, const RouteBufs& rb,
-                         cudaStream_t s) {
+                         cudaStream_t s, int pdl = 0) {
     const Dims& d = h->d;
     TcMaps maps{};
     moe_status st = make_map(&maps.b_x, x, (uint64_t)T, d.H, 16);
@@ -420,7 +420,7 @@ moe_status run_tc_router(moe_layer* h, const void* x, int T, const RouteBufs& rb
     a.sync = h->sync_router;
     a.st = h->status(); a.wait_limit_ns = h->wait_limit_ns; a.inject_stuck = 0;
     const int tiles = (T + kNarrow - 1) / kNarrow * ((d.E / 128 + 1) / 2);
-    CUDA_TRY(launch_tc_experts(maps, a, kNarrow, std::min(tiles, h->num_sms), s));
+    CUDA_TRY(launch_tc_experts(maps, a, kNarrow, std::min(tiles, h->num_sms), s, pdl));
     return MOE_OK;
 }
 
@@ -535,6 +535,10 @@ moe_status run_layer(moe_layer* h, const void* x, const void* residual, void* y,
     // every SM while the router waited).  CUDA cores: optionally a second stream.
     const bool merged = tc && d.Is > 0;
     const bool side = !merged && h->shared_stream && d.Is > 0;
+    // Programmatic dependent launch is off on this path: measured at 4096 tokens it
+    // cost 7 us per layer (the persistent expert kernel's early CTAs took SMs from the
+    // permutation kernel); the few-token path uses it.
+    const int pdl = 0;
 
     if (side && !h->rms_w) {     // the shared expert needs only x: start it right away
         CUDA_TRY(cudaEventRecord(h->ev_fork, s));
@@ -552,12 +556,12 @@ moe_status run_layer(moe_layer* h, const void* x, const void* residual, void* y,
     {
         KernelScope ks(h, MOE_KERNEL_ROUTER, s);
         if (tc_route) {
-            moe_status st = run_tc_router(h, x, T, rb, s);
+            moe_status st = run_tc_router(h, x, T, rb, s, pdl);
             if (st != MOE_OK) return st;
         }
         CUDA_TRY(launch_router(h->dtype, x, h->w_router, h->rms_w, h->cfg.rms_eps, h->x_norm,
                                fused_permute, xp_copy, d, T, tb, rb, 1, width, h->max_units,
-                               tc_route, h->status(), s));
+                               tc_route, h->status(), s, pdl));
     }
     if (side && h->rms_w) {      // with a pre-norm it needs the router's normalised x
         CUDA_TRY(cudaEventRecord(h->ev_fork, s));
@@ -568,7 +572,7 @@ moe_status run_layer(moe_layer* h, const void* x, const void* residual, void* y,
     }
     if (!fused_permute) {
         KernelScope ks(h, MOE_KERNEL_PERMUTE, s);
-        CUDA_TRY(launch_permute(h->dtype, x_in, xp_copy, d, T, tb, rb, s));
+        CUDA_TRY(launch_permute(h->dtype, x_in, xp_copy, d, T, tb, rb, s, pdl));
     }
     const int S = T * d.k;
     if (tc) {
@@ -597,12 +601,12 @@ moe_status run_layer(moe_layer* h, const void* x, const void* residual, void* y,
         const int grid = std::min(tiles, h->num_sms);
         {
             KernelScope ks(h, MOE_KERNEL_EXPERTS, s);
-            CUDA_TRY(launch_tc_experts(maps, a, width, grid, s));
+            CUDA_TRY(launch_tc_experts(maps, a, width, grid, s, pdl));
         }
         if (!h->fuse) {
             a.phases = 2;
             KernelScope ks(h, MOE_KERNEL_EXPERTS, s);
-            CUDA_TRY(launch_tc_experts(maps, a, width, grid, s));
+            CUDA_TRY(launch_tc_experts(maps, a, width, grid, s, pdl));
         }
         h->inject_stuck = 0;
     } else {
@@ -627,7 +631,7 @@ moe_status run_layer(moe_layer* h, const void* x, const void* residual, void* y,
     {
         KernelScope ks(h, MOE_KERNEL_COMBINE, s);
         CUDA_TRY(launch_combine(h->dtype, h->obuf, d.Is > 0 ? h->sbuf : nullptr, residual, y,
-                                rb.topk_w, rb.token_slot, d, T, s));
+                                rb.topk_w, rb.token_slot, d, T, s, pdl));
     }
     h->last_T = T;
     return MOE_OK;

@@ -394,6 +394,8 @@ __global__ void __launch_bounds__(kThreads)
 permute_kernel(const Tin* __restrict__ x_in, Tin* __restrict__ xp, Dims d, int T, int tb,
                RouteBufs rb) {
     extern __shared__ uint32_t sm[];
+    grid_dependency_wait();          // the router's histograms and offsets
+    grid_dependents_launch();
     permute_block<Tin>(x_in, xp, d, T, tb, blockIdx.x, blockIdx.y, gridDim.y, rb, sm);
 }
 
@@ -450,20 +452,27 @@ cudaError_t launch_router(int dtype, const void* x, const void* w_router, const 
 }
 
 cudaError_t launch_permute(int dtype, const void* x_in, void* xp, const Dims& d, int T, int tb,
-                           const RouteBufs& rb, cudaStream_t s) {
+                           const RouteBufs& rb, cudaStream_t s, int pdl) {
     if (T <= 0) return cudaSuccess;
     if (tb > 128) return cudaErrorInvalidValue;
     const int nblocks = (T + tb - 1) / tb;
     const int split = std::max(1, std::min(16, (2 * 148 + nblocks - 1) / nblocks));   // >= 2 CTAs/SM
     const size_t smem = (size_t)d.E * 4 * sizeof(uint32_t) + (size_t)tb * d.k * sizeof(int);
-    dim3 grid(nblocks, split);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nblocks, split);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
     if (dtype == 0)
-        permute_kernel<float><<<grid, kThreads, smem, s>>>((const float*)x_in, (float*)xp, d, T,
-                                                          tb, rb);
-    else
-        permute_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(
-            (const __nv_bfloat16*)x_in, (__nv_bfloat16*)xp, d, T, tb, rb);
-    return cudaGetLastError();
+        return cudaLaunchKernelEx(&cfg, permute_kernel<float>, (const float*)x_in, (float*)xp, d,
+                                  T, tb, rb);
+    return cudaLaunchKernelEx(&cfg, permute_kernel<__nv_bfloat16>, (const __nv_bfloat16*)x_in,
+                              (__nv_bfloat16*)xp, d, T, tb, rb);
 }
 
 }  // namespace moe
