@@ -86,7 +86,7 @@ moe_status make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
 }
 
 constexpr int kRouteBlock = 16;      // routing block with CUDA-core logits (T < 256)
-constexpr int kRouteBlockWide = 64;  // routing block after tensor-core logits
+constexpr int kRouteBlockWide = 128; // routing block after tensor-core logits
 constexpr int kNarrow = 32, kWide = 256;
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }

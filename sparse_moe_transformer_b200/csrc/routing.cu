@@ -31,7 +31,6 @@ constexpr int kEG = 2;              // experts per logits CTA: 4 warps per exper
 constexpr int kMaxTB = 16;          // tokens per logits CTA
 constexpr int kMaxE = 1024;
 constexpr int kMaxK = 16;
-constexpr int kChunk = 32;          // routing blocks per scan chunk
 
 // VEC consecutive elements as fp32 (VEC * sizeof(T) == 16: one vector load).
 template <typename T, int VEC>
@@ -170,6 +169,11 @@ __device__ void permute_block(const Tin* __restrict__ x_in, Tin* __restrict__ xp
     }
 }
 
+// Part sums of the column scan live after the chunk rows in dynamic shared memory.
+__device__ __forceinline__ int* scan_tmp_big(uint8_t* dyn, int rows, int E) {
+    return reinterpret_cast<int*>(dyn) + (size_t)rows * E;
+}
+
 struct RouterArgs {
     const void* x;
     const void* w_router;
@@ -181,6 +185,7 @@ struct RouterArgs {
     Dims d;
     int T, tb, tt;       // routing block, tokens per CTA group
     int do_scan, unit_width, max_units, select_only;
+    int scan_rows;       // histogram rows per scan chunk
     RouteBufs rb;
     DeviceStatus st;
 };
@@ -324,26 +329,59 @@ __global__ void __launch_bounds__(kThreads) router_kernel(RouterArgs a) {
         __threadfence();
     }
     const int nrb = (a.T + a.tb - 1) / a.tb;              // routing blocks
-    int* chunk = reinterpret_cast<int*>(dyn);          // [kChunk][E] histogram rows
+    // Column scan of the [nrb][E] histograms: block_off[b][e] = sum_{b' < b} hist[b'][e].
+    // A chunk of rows is loaded with many loads in flight; P = kThreads / E threads
+    // share an expert's column (two passes over the chunk, then a fix-up).
+    int* chunk = reinterpret_cast<int*>(dyn);          // [cb][E] histogram rows
+    const int cb = a.scan_rows;                        // rows per chunk (fits the smem)
+    const int P = max(1, kThreads / E);                // threads per expert column
+    int* psum = scan_tmp_big(dyn, cb, E);              // [P][E] part sums
     for (int e = tid; e < E; e += kThreads) hist[e] = 0;    // running count per expert
 #pragma unroll 1
-    for (int b0 = 0; b0 < nrb; b0 += kChunk) {
-        const int nb = min(kChunk, nrb - b0);
+    for (int b0 = 0; b0 < nrb; b0 += cb) {
+        const int nb = min(cb, nrb - b0);
         __syncthreads();
-#pragma unroll 4
-        for (int i = tid; i < nb * E; i += kThreads) {
-            chunk[i] = __ldcg(rb.block_hist + (size_t)b0 * E + i);
-            rb.block_hist[(size_t)b0 * E + i] = 0;
+        const int n = nb * E;
+        const int* src = rb.block_hist + (size_t)b0 * E;
+#pragma unroll 1
+        for (int i0 = tid; i0 < n; i0 += 16 * kThreads) {
+            int v[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int i = i0 + j * kThreads;
+                v[j] = i < n ? __ldcg(src + i) : 0;
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int i = i0 + j * kThreads;
+                if (i < n) { chunk[i] = v[j]; rb.block_hist[(size_t)b0 * E + i] = 0; }
+            }
         }
         __syncthreads();
-        for (int e = tid; e < E; e += kThreads) {
+        const int e = tid % E, part = tid / E;
+        const int per = (nb + P - 1) / P;
+        const int j0 = min(nb, part * per), j1 = min(nb, j0 + per);
+        if (tid < P * E) {
+            int sum = 0;
+#pragma unroll 8
+            for (int j = j0; j < j1; ++j) sum += chunk[j * E + e];
+            psum[part * E + e] = sum;
+        }
+        __syncthreads();
+        if (tid < P * E) {
             int run = hist[e];
-#pragma unroll 1
-            for (int j = 0; j < nb; ++j) {
+            for (int q = 0; q < part; ++q) run += psum[q * E + e];
+#pragma unroll 8
+            for (int j = j0; j < j1; ++j) {
                 rb.block_off[(size_t)(b0 + j) * E + e] = run;
                 run += chunk[j * E + e];
             }
-            hist[e] = run;
+        }
+        __syncthreads();
+        if (tid < E) {
+            int tot = hist[tid];
+            for (int q = 0; q < P; ++q) tot += psum[q * E + tid];
+            hist[tid] = tot;
         }
     }
     __syncthreads();
@@ -438,10 +476,14 @@ cudaError_t launch_router(int dtype, const void* x, const void* w_router, const 
     if (d.E > kMaxE || d.k > kMaxK || tb > 128) return cudaErrorInvalidValue;
     const int tt = select_only ? kWarps : kMaxTB;   // select: one token per warp
     if (!select_only && tb != kMaxTB) return cudaErrorInvalidValue;
+    const int nrb = (T + tb - 1) / tb;
+    const int parts = std::max(1, kThreads / d.E);
+    // scan chunk: up to 48 KB of histogram rows (all of them when they fit)
+    const int scan_rows = std::max(1, std::min(nrb, (48 * 1024) / (d.E * 4)));
     RouterArgs a{x, w_router, rms_w, rms_eps, x_norm, permute, xp, d, T, tb, tt, do_scan,
-                 unit_width, max_units, select_only, rb, ds};
+                 unit_width, max_units, select_only, scan_rows, rb, ds};
     dim3 grid(select_only ? 1 : (d.E + kEG - 1) / kEG, (T + tt - 1) / tt);
-    size_t smem = (size_t)kChunk * d.E * 4;                                        // scan chunk
+    size_t smem = do_scan ? (size_t)(scan_rows + parts) * d.E * 4 : 0;            // scan chunk
     smem = std::max(smem, (size_t)2 * kMaxE * 4 + (size_t)d.E * 16 + (size_t)tb * d.k * 4);
     if (smem > 200 * 1024) return cudaErrorInvalidValue;
     if (dtype == 0)
