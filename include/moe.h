@@ -166,8 +166,9 @@ moe_status moe_set_option(moe_handle h, moe_option opt, int64_t value);
 typedef enum {
     MOE_KERNEL_ROUTER = 0,     /* logits, Top-k, weights, histogram, scan            */
     MOE_KERNEL_PERMUTE = 1,    /* gather of token rows into expert-contiguous order  */
-    MOE_KERNEL_EXPERTS = 2,    /* routed expert GEMMs (gate/up + SiLU*up, down)      */
-    MOE_KERNEL_SHARED = 3,     /* shared expert GEMMs                                */
+    MOE_KERNEL_EXPERTS = 2,    /* expert GEMMs (gate/up + SiLU*up, down); on tensor
+                                  cores the shared expert's tiles run in them too   */
+    MOE_KERNEL_SHARED = 3,     /* shared expert GEMMs on CUDA cores (fp32 layers)    */
     MOE_KERNEL_COMBINE = 4,    /* weighted combine + shared + residual               */
     MOE_KERNEL_CLASSES = 5
 } moe_kernel_class;

@@ -517,17 +517,11 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
     }
 }
 
-// Two entry points with one body, so profiles tell the routed experts (grouped,
-// device-built unit list) from the dense shared expert.
+// Two entry points with one body, so profiles tell the expert GEMMs (grouped
+// routed experts, with the shared expert's dense tiles) from the router logits.
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_routed_experts_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
-    tc_experts_body<BN>(maps, a);
-}
-
-template <int BN>
-__global__ void __launch_bounds__(kThreads, 1)
-tc_shared_expert_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     tc_experts_body<BN>(maps, a);
 }
 
@@ -544,10 +538,6 @@ cudaError_t launch_width(const TcMaps& maps, const TcArgs& a, int grid, int pdl,
         cudaError_t e = cudaFuncSetAttribute(tc_routed_experts_kernel<BN>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              TcCfg<BN>::kSmem);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(tc_shared_expert_kernel<BN>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     TcCfg<BN>::kSmem);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(tc_router_logits_kernel<BN>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -566,7 +556,6 @@ cudaError_t launch_width(const TcMaps& maps, const TcArgs& a, int grid, int pdl,
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
     if (a.phases == 4) return cudaLaunchKernelEx(&cfg, tc_router_logits_kernel<BN>, maps, a);
-    if (a.dense_T > 0) return cudaLaunchKernelEx(&cfg, tc_shared_expert_kernel<BN>, maps, a);
     return cudaLaunchKernelEx(&cfg, tc_routed_experts_kernel<BN>, maps, a);
 }
 

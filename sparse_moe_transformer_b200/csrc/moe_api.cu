@@ -424,42 +424,19 @@ moe_status run_tc_router(moe_layer* h, const void* x, int T, const RouteBufs& rb
     return MOE_OK;
 }
 
+// CUDA-core shared expert (fp32 layers and forced CUDA-core runs); the tensor-core
+// paths run the shared expert's tiles inside their expert kernel.
 moe_status run_shared(moe_layer* h, const void* x_in, int T, cudaStream_t s) {
     const Dims& d = h->d;
     if (!d.Is) return MOE_OK;
-    if (h->tc_ok && !h->force_simt) {
-        TcMaps maps = h->shared_maps;
-        moe_status st = make_map(&maps.b_x, x_in, (uint64_t)T, d.H, 16);
-        if (st != MOE_OK) return st;
-        const int width = choose_width(h, T);
-        TcArgs a{};
-        a.w_gu = h->ws_gate; a.w_down = h->ws_down;
-        a.H = d.H; a.I = d.Is; a.phases = h->fuse ? 3 : 1;
-        a.dense_T = T; a.unit_width = width;
-        a.units = nullptr; a.n_units = nullptr;
-        a.sync = h->sync_shared; a.hbuf = h->hs; a.out = h->sbuf;
-        a.st = h->status(); a.wait_limit_ns = h->wait_limit_ns; a.inject_stuck = 0;
-        const int units = (T + width - 1) / width;
-        const int tiles = units * (d.Is / 128 + (d.H / 128 + 1) / 2);
-        {
-            KernelScope ks(h, MOE_KERNEL_SHARED, s);
-            CUDA_TRY(launch_tc_experts(maps, a, width, std::min(tiles, h->num_sms), s));
-        }
-        if (!h->fuse) {
-            a.phases = 2;
-            KernelScope ks(h, MOE_KERNEL_SHARED, s);
-            CUDA_TRY(launch_tc_experts(maps, a, width, std::min(tiles, h->num_sms), s));
-        }
-    } else {
-        {
-            KernelScope ks(h, MOE_KERNEL_SHARED, s);
-            CUDA_TRY(launch_simt_gate_up(h->dtype, x_in, h->ws_gate, h->ws_up, h->tc_ok, nullptr,
-                                         nullptr, T, d.H, d.Is, h->hs, s));
-        }
+    {
         KernelScope ks(h, MOE_KERNEL_SHARED, s);
-        CUDA_TRY(launch_simt_down(h->dtype, h->hs, h->ws_down, h->tc_ok, nullptr, nullptr, T,
-                                  d.H, d.Is, h->sbuf, s));
+        CUDA_TRY(launch_simt_gate_up(h->dtype, x_in, h->ws_gate, h->ws_up, h->tc_ok, nullptr,
+                                     nullptr, T, d.H, d.Is, h->hs, s));
     }
+    KernelScope ks(h, MOE_KERNEL_SHARED, s);
+    CUDA_TRY(launch_simt_down(h->dtype, h->hs, h->ws_down, h->tc_ok, nullptr, nullptr, T, d.H,
+                              d.Is, h->sbuf, s));
     return MOE_OK;
 }
 
