@@ -108,7 +108,10 @@ moe_status moe_route(moe_handle h, const void* x, int T, int32_t* topk_idx,
  * [T][k]) receive the routing the call used.  T == 0 is a no-op.
  * Few tokens (T * k <= 1024, bf16, H a multiple of 256 up to 1024, k <= 8) run
  * as router + one expert kernel (the shared expert's blocks among its tiles) +
- * combine, each kernel a programmatic dependent of the one before.  Larger calls
+ * combine, each kernel a programmatic dependent of the one before.  Up to 64
+ * tokens with 128 experts and no pre-norm, the router is one CTA that forms the
+ * logits on the tensor cores (fp32 accumulate), so its routing can differ from
+ * moe_route's CUDA-core logits by fp32 rounding (weights) and at exact near-ties.  Larger calls
  * run router, permutation, one grouped expert GEMM launch (the shared expert's
  * tiles among the routed experts') and combine.
  */

@@ -139,21 +139,24 @@ simt_down_kernel(const T* __restrict__ h, const T* __restrict__ wd,
 // Down (src1 == nullptr): pair index (e, mt2, kb), member = row block 2 mt2 + member.
 __global__ void __launch_bounds__(256)
 pack_tiles_kernel(const uint4* __restrict__ src0, const uint4* __restrict__ src1,
-                  uint4* __restrict__ dst, int E, int R, int C, size_t total) {
+                  uint4* __restrict__ dst, int E, int R, int C, int kpair, size_t total) {
     const int MT = R / 128, KB = C / 64;
-    const int NB = src1 ? MT : (MT + 1) / 2;      // row blocks (or block pairs) per expert
+    const int NB = (src1 || kpair) ? MT : (MT + 1) / 2;   // row blocks (or block pairs) per expert
+    const int KP = kpair ? KB / 2 : KB;                     // pairs along the columns
     for (size_t v = blockIdx.x * (size_t)blockDim.x + threadIdx.x; v < total;
          v += (size_t)gridDim.x * blockDim.x) {
         const int r = (int)((v >> 3) & 127);
         const int c8 = (int)(v & 7) ^ (r & 7);
         size_t rest = v >> 10;
         const int member = (int)(rest & 1); rest >>= 1;
-        const int kb = (int)(rest % KB); rest /= KB;
+        int kb = (int)(rest % KP); rest /= KP;
         const int nb = (int)(rest % NB);
         const int e = (int)(rest / NB);
         const uint4* src = src0;
         int mt = nb;
-        if (src1) {
+        if (kpair) {
+            kb = 2 * kb + member;
+        } else if (src1) {
             src = member ? src1 : src0;
         } else {
             mt = 2 * nb + member;
@@ -338,7 +341,16 @@ cudaError_t launch_pack_tiles(const void* src0, const void* src1, void* dst, int
     const size_t total = (size_t)E * NB * (C / 64) * 2 * 1024;     // 16-byte vectors
     const int grid = (int)std::min<size_t>((total + 255) / 256, 148 * 32);
     pack_tiles_kernel<<<grid, 256, 0, s>>>((const uint4*)src0, (const uint4*)src1, (uint4*)dst,
-                                           E, R, C, total);
+                                           E, R, C, 0, total);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_kpairs(const void* src, void* dst, int R, int C, cudaStream_t s) {
+    if (R % 128 || C % 128) return cudaErrorInvalidValue;
+    const size_t total = (size_t)(R / 128) * (C / 128) * 2 * 1024;  // 16-byte vectors
+    const int grid = (int)std::min<size_t>((total + 255) / 256, 148 * 32);
+    pack_tiles_kernel<<<grid, 256, 0, s>>>((const uint4*)src, nullptr, (uint4*)dst, 1, R, C, 1,
+                                           total);
     return cudaGetLastError();
 }
 

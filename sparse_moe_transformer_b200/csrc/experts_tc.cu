@@ -533,8 +533,8 @@ tc_router_logits_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
 
 template <int BN>
 cudaError_t launch_width(const TcMaps& maps, const TcArgs& a, int grid, int pdl, cudaStream_t s) {
-    static bool configured = false;   // per process; the attribute is per function
-    if (!configured) {
+    static bool configured[16] = {};    // per device: the attribute is set per device
+    if (first_use_on_device(configured)) {
         cudaError_t e = cudaFuncSetAttribute(tc_routed_experts_kernel<BN>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              TcCfg<BN>::kSmem);
@@ -543,7 +543,6 @@ cudaError_t launch_width(const TcMaps& maps, const TcArgs& a, int grid, int pdl,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      TcCfg<BN>::kSmem);
         if (e != cudaSuccess) return e;
-        configured = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);

@@ -47,6 +47,16 @@ struct RouteBufs {
     int32_t* tickets;     // [T / 8 + 1] arrival counters (self-resetting)
 };
 
+// A launcher's once-per-device set-up (kernel attributes are set per device):
+// true the first time it is asked for the current device.
+inline bool first_use_on_device(bool (&done)[16]) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return true;
+    if (done[dev]) return false;
+    done[dev] = true;
+    return true;
+}
+
 // ---------------------------------------------------------------- launchers
 // Router: logits (fp32 accumulate), optional fused pre-RMSNorm, Top-k with the
 // lower-index tie rule, renormalised weights, per-block histograms and (when
@@ -61,6 +71,22 @@ cudaError_t launch_router(int dtype, const void* x, const void* w_router, const 
                           int T, int tb, const RouteBufs& rb, int do_scan, int unit_width,
                           int max_units, int select_only, const DeviceStatus& st,
                           cudaStream_t s, int pdl = 0);
+
+// One-CTA tensor-core router for a handful of tokens (bf16, no pre-norm, 128
+// experts, T <= 64): W_r packed as k-pairs (launch_pack_kpairs), x by a TMA map
+// with 64 x round16(T) boxes.  Writes topk_idx / topk_w.
+struct RouterTcArgs {
+    const void* w_router_kp;
+    int32_t* topk_idx;
+    float* topk_w;
+    int H, k, T;
+    DeviceStatus st;
+    uint64_t wait_limit_ns;
+};
+bool router_tc_supported(int E, int H, int k, int T);
+// pdl: launch as a programmatic dependent of the previous kernel in the stream.
+cudaError_t launch_router_tc(const CUtensorMap& xmap, const RouterTcArgs& a, int pdl,
+                             cudaStream_t s);
 
 // Expert-contiguous order of the token rows: fills token_slot / slot_token /
 // slot_expert, and gathers the rows into xp unless xp is null.
@@ -105,6 +131,10 @@ __host__ __device__ inline size_t packed_down_elems(int E, int H, int I) {
 // src1 != nullptr, else down row-block pairs (dst must be zeroed when R / 128 is odd).
 cudaError_t launch_pack_tiles(const void* src0, const void* src1, void* dst, int E, int R, int C,
                               cudaStream_t s);
+// Pack a [R][C] matrix (bf16) as k-pairs: pair (mt, p) = tile (mt, 2p) then tile
+// (mt, 2p + 1), pairs ordered mt then p (R % 128 == 0, C % 128 == 0): one 32 KB
+// bulk copy carries 128 columns of one 128-row block.
+cudaError_t launch_pack_kpairs(const void* src, void* dst, int R, int C, cudaStream_t s);
 
 
 // CUDA-core expert kernels (exact fp32 accumulate; any shape).

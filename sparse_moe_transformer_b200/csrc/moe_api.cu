@@ -110,6 +110,7 @@ struct moe_layer {
     void *w_router = nullptr, *w_gate = nullptr, *w_up = nullptr, *w_down = nullptr;
     void *ws_gate = nullptr, *ws_up = nullptr, *ws_down = nullptr, *rms_w = nullptr;
     void* w_router_packed = nullptr;   // tensor-core router (E % 128 == 0, no pre-norm)
+    void* w_router_kp = nullptr;       // W_r as k-pairs: one-CTA router for a few tokens
     // workspace
     int max_T = 0;
     int max_units = 0;
@@ -160,6 +161,14 @@ moe_status pack_weight(void** dst, const void* src0, const void* src1, int E, in
     CUDA_TRY(cudaMalloc(dst, bytes));
     CUDA_TRY(cudaMemset(*dst, 0, bytes));
     CUDA_TRY(launch_pack_tiles(src0, src1, *dst, E, R, C, 0));
+    CUDA_TRY(cudaStreamSynchronize(0));
+    return MOE_OK;
+}
+
+// W_r [R][C] as k-pairs (launch_pack_kpairs) for the one-CTA tensor-core router.
+moe_status pack_kpair_weight(void** dst, const void* src, int R, int C) {
+    CUDA_TRY(cudaMalloc(dst, (size_t)R * C * 2));
+    CUDA_TRY(launch_pack_kpairs(src, *dst, R, C, 0));
     CUDA_TRY(cudaStreamSynchronize(0));
     return MOE_OK;
 }
@@ -287,6 +296,8 @@ moe_status moe_create(const moe_config* cfg, int device, const void* w_router, c
         chk(pack_weight(&h->w_down, w_down, nullptr, (int)E, (int)H, (int)I));
         if (E % 128 == 0 && !rms_weight)
             chk(pack_weight(&h->w_router_packed, w_router, nullptr, 1, (int)E, (int)H));
+        if (!rms_weight && router_tc_supported((int)E, (int)H, c.top_k, 1))
+            chk(pack_kpair_weight(&h->w_router_kp, w_router, (int)E, (int)H));
         if (Is) {
             chk(pack_weight(&h->ws_gate, ws_gate, ws_up, 1, (int)Is, (int)H));
             chk(pack_weight(&h->ws_down, ws_down, nullptr, 1, (int)H, (int)Is));
@@ -454,9 +465,21 @@ moe_status run_layer_fused(moe_layer* h, const void* x, const void* residual, vo
     const int pdl = h->timing ? 0 : 1;
     {
         KernelScope ks(h, MOE_KERNEL_ROUTER, s);
-        CUDA_TRY(launch_router(h->dtype, x, h->w_router, h->rms_w, h->cfg.rms_eps, h->x_norm, 0,
-                               nullptr, d, T, kRouteBlock, rb, 0, kNarrow, h->max_units, 0,
-                               h->status(), s, pdl));
+        if (h->w_router_kp && router_tc_supported(d.E, d.H, d.k, T)) {
+            // a handful of tokens: one CTA forms the logits on the tensor cores
+            CUtensorMap xmap;
+            moe_status st = make_map(&xmap, x, (uint64_t)T, d.H, (T + 15) / 16 * 16);
+            if (st != MOE_OK) return st;
+            RouterTcArgs ra{};
+            ra.w_router_kp = h->w_router_kp; ra.topk_idx = rb.topk_idx; ra.topk_w = rb.topk_w;
+            ra.H = d.H; ra.k = d.k; ra.T = T;
+            ra.st = h->status(); ra.wait_limit_ns = h->wait_limit_ns;
+            CUDA_TRY(launch_router_tc(xmap, ra, pdl, s));
+        } else {
+            CUDA_TRY(launch_router(h->dtype, x, h->w_router, h->rms_w, h->cfg.rms_eps, h->x_norm,
+                                   0, nullptr, d, T, kRouteBlock, rb, 0, kNarrow, h->max_units,
+                                   0, h->status(), s, pdl));
+        }
     }
     const int S = T * d.k;
     {
@@ -774,7 +797,8 @@ moe_status moe_destroy(moe_handle h) {
     for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
     free_workspace(h);
     void* bufs[] = {h->w_router, h->w_gate, h->w_up,  h->w_down,  h->ws_gate,
-                    h->ws_up,    h->ws_down, h->rms_w, h->err_dev, h->w_router_packed};
+                    h->ws_up,    h->ws_down, h->rms_w, h->err_dev, h->w_router_packed,
+                    h->w_router_kp};
     for (void* p : bufs)
         if (p) cudaFree(p);
     if (h->err_host) cudaFreeHost(h->err_host);

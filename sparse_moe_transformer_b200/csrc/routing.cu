@@ -31,6 +31,7 @@ constexpr int kEG = 2;              // experts per logits CTA: 4 warps per exper
 constexpr int kMaxTB = 16;          // tokens per logits CTA
 constexpr int kMaxE = 1024;
 constexpr int kMaxK = 16;
+constexpr int kMaxRouterSmem = 200 * 1024;   // dynamic shared memory of a router launch
 
 // VEC consecutive elements as fp32 (VEC * sizeof(T) == 16: one vector load).
 template <typename T, int VEC>
@@ -440,14 +441,19 @@ permute_kernel(const Tin* __restrict__ x_in, Tin* __restrict__ xp, Dims d, int T
 template <typename Tin, int VEC>
 cudaError_t launch_router_t(const RouterArgs& a, dim3 grid, size_t smem, int pdl, cudaStream_t s) {
     const int epl = (a.d.E + 31) / 32;
-    auto go = [&](auto kernel) -> cudaError_t {
-        static int allowed = 0;          // per kernel instance: dynamic smem already allowed
-        if ((int)smem > allowed) {
+    // Every instance may take up to kMaxRouterSmem bytes of dynamic shared memory; the
+    // attribute is set once per instance (the three instances share one signature, so
+    // a per-call "already allowed" record could not tell them apart).
+    static bool configured[16] = {};    // per device: the attribute is set per device
+    if (first_use_on_device(configured)) {
+        for (auto kernel : {router_kernel<Tin, VEC, 4>, router_kernel<Tin, VEC, 8>,
+                            router_kernel<Tin, VEC, 32>}) {
             cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)smem);
+                                                 kMaxRouterSmem);
             if (e != cudaSuccess) return e;
-            allowed = (int)smem;
         }
+    }
+    auto go = [&](auto kernel) -> cudaError_t {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = grid;
         cfg.blockDim = dim3(kThreads);
@@ -485,7 +491,7 @@ cudaError_t launch_router(int dtype, const void* x, const void* w_router, const 
     dim3 grid(select_only ? 1 : (d.E + kEG - 1) / kEG, (T + tt - 1) / tt);
     size_t smem = do_scan ? (size_t)(scan_rows + parts) * d.E * 4 : 0;            // scan chunk
     smem = std::max(smem, (size_t)2 * kMaxE * 4 + (size_t)d.E * 16 + (size_t)tb * d.k * 4);
-    if (smem > 200 * 1024) return cudaErrorInvalidValue;
+    if (smem > (size_t)kMaxRouterSmem) return cudaErrorInvalidValue;
     if (dtype == 0)
         return d.H % 4 == 0 ? launch_router_t<float, 4>(a, grid, smem, pdl, s)
                             : launch_router_t<float, 1>(a, grid, smem, pdl, s);
