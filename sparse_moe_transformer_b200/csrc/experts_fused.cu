@@ -1,5 +1,6 @@
-// experts_fused.cu -- routed SwiGLU experts for few tokens (decode), one tile =
-// one expert's tokens x one 128-feature block of the intermediate dimension.
+// experts_fused.cu -- routed and shared SwiGLU experts for few tokens (decode),
+// one tile = one expert's tokens (or the shared expert's) x one 128-feature block
+// of the intermediate dimension.
 //
 // Each expert is down(SiLU(gate x) * up x) (page "print(model) Qwen3-TTS",
 // SwiGLU section).  Splitting the intermediate dimension I into 128-feature
@@ -11,12 +12,13 @@
 // outputs.  Tiles never wait for one another; each writes an fp32 partial
 // o_part[b][slot][H] and the combine sums the blocks in fixed order.
 //
-// The token lists come straight from the router's Top-k: every CTA builds the
-// same expert-ordered unit list from topk_idx in shared memory (tokens of one
-// expert in token order, split into runs of at most kBN), so no permutation
-// pass or global scan runs before this kernel.  The shared expert's tiles come
-// first in the tile list; they need no routing and, when the layer input is
-// used as is, start while the router still runs (programmatic dependent launch).
+// The token lists come straight from the router's Top-k: every CTA counts the
+// selections per expert in shared memory and finds each of its own tiles' expert
+// and rows with ballots (the rows of an expert in token order, cut into units of
+// at most kBN), so no permutation pass or global scan runs before this kernel.
+// CTA b takes tiles b, b + G, b + 2G, ... of [shared-expert tiles | routed tiles];
+// the shared tiles need no routing and, when the layer input is used as is,
+// start while the router still runs (programmatic dependent launch).
 //
 // Warp roles: warp 0 schedules tiles and streams weights (contiguous bulk copies
 // of pre-swizzled tile pairs, nothing else, so it runs ahead by the full stage

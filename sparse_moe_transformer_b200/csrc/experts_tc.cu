@@ -21,13 +21,14 @@
 // The kernel is persistent: CTAs take tiles from a global counter, gate/up tiles
 // first, then down tiles.  A launch may carry a second, dense problem -- the
 // shared expert over every token -- whose tiles interleave as [routed gate/up |
-// shared gate/up | routed down | shared down].  When both phases run in one launch, a down tile of a
-// unit waits (bounded by a time limit) until the unit's gate/up tiles have
-// published their h rows; every gate/up tile is taken before any down tile and
-// never waits, so the wait always ends.  (Ordering tiles in waves of units --
-// each wave's gate/up then down tiles -- was measured slower: down tiles then
-// hold SMs idle while their wave's gate/up tiles still stream.)  Every wait in the kernel is bounded; a
-// wait that runs out records MOE_ERR_TIMEOUT and the CTA drains and exits.
+// shared gate/up | routed down | shared down].  When both phases run in one
+// launch, a down tile of a unit waits (bounded by a time limit) until the unit's
+// gate/up tiles have published their h rows; every gate/up tile is taken before
+// any down tile and never waits, so the wait always ends.  (Ordering tiles in
+// waves of units -- each wave's gate/up then down tiles -- was measured slower:
+// down tiles then hold SMs idle while their wave's gate/up tiles still stream.)
+// Every wait in the kernel is bounded; a wait that runs out records
+// MOE_ERR_TIMEOUT and the CTA drains and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
