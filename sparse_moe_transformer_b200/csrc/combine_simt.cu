@@ -26,7 +26,7 @@ __global__ void __launch_bounds__(128)
 combine_kernel(const T* __restrict__ o, const T* __restrict__ sh, const T* res, T* y,
                const float* __restrict__ topk_w,
                const int32_t* __restrict__ token_slot, int H, int k) {
-    grid_dependency_wait();          // expert outputs of the previous kernel
+    grid_dependency_wait();          // expert outputs (no-op unless a dependent launch)
     grid_dependents_launch();
     const int t = blockIdx.x;
     __shared__ int slot[16];

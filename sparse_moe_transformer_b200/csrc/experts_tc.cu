@@ -204,8 +204,9 @@ __device__ __forceinline__ void tc_experts_body(const TcMaps& maps, const TcArgs
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    // launched as a programmatic dependent: the set-up above overlapped the previous
-    // kernel; from here on its results (units, activations) are read
+    // when launched as a programmatic dependent, the set-up above overlaps the previous
+    // kernel and its results (units, activations) are read only from here on (a no-op
+    // otherwise)
     grid_dependency_wait();
     grid_dependents_launch();
 

@@ -433,7 +433,7 @@ __global__ void __launch_bounds__(kThreads)
 permute_kernel(const Tin* __restrict__ x_in, Tin* __restrict__ xp, Dims d, int T, int tb,
                RouteBufs rb) {
     extern __shared__ uint32_t sm[];
-    grid_dependency_wait();          // the router's histograms and offsets
+    grid_dependency_wait();          // the router's histograms (no-op unless a dependent launch)
     grid_dependents_launch();
     permute_block<Tin>(x_in, xp, d, T, tb, blockIdx.x, blockIdx.y, gridDim.y, rb, sm);
 }
