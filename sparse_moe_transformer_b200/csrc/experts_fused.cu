@@ -512,13 +512,13 @@ bool fused_supported(int H, int I, int Is, int E, int k, int S) {
 cudaError_t launch_fused_experts(const FusedArgs& a, int grid, int pdl, cudaStream_t s) {
     if (grid <= 0) return cudaSuccess;
     if (!fused_supported(a.H, a.I, a.Is, a.E, a.k, a.T * a.k)) return cudaErrorInvalidValue;
-    static bool configured[16] = {};    // per device: the attribute is set per device
-    if (first_use_on_device(configured)) {
-        cudaError_t e = cudaFuncSetAttribute(tc_fused_experts_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             SmemLayout::kTotal);
-        if (e != cudaSuccess) return e;
-    }
+    static std::once_flag configured[16];    // the attribute is set per device
+    cudaError_t e = once_per_device(configured, [] {
+        return cudaFuncSetAttribute(tc_fused_experts_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    SmemLayout::kTotal);
+    });
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);

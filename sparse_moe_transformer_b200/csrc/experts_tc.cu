@@ -535,17 +535,18 @@ tc_router_logits_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
 
 template <int BN>
 cudaError_t launch_width(const TcMaps& maps, const TcArgs& a, int grid, int pdl, cudaStream_t s) {
-    static bool configured[16] = {};    // per device: the attribute is set per device
-    if (first_use_on_device(configured)) {
-        cudaError_t e = cudaFuncSetAttribute(tc_routed_experts_kernel<BN>,
+    static std::once_flag configured[16];    // the attribute is set per device
+    cudaError_t e = once_per_device(configured, [] {
+        cudaError_t r = cudaFuncSetAttribute(tc_routed_experts_kernel<BN>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              TcCfg<BN>::kSmem);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(tc_router_logits_kernel<BN>,
+        if (r == cudaSuccess)
+            r = cudaFuncSetAttribute(tc_router_logits_kernel<BN>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      TcCfg<BN>::kSmem);
-        if (e != cudaSuccess) return e;
-    }
+        return r;
+    });
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace moe {
 
 // device-side error codes (same values as the public moe_status)
@@ -47,14 +49,16 @@ struct RouteBufs {
     int32_t* tickets;     // [T / 8 + 1] arrival counters (self-resetting)
 };
 
-// A launcher's once-per-device set-up (kernel attributes are set per device):
-// true the first time it is asked for the current device.
-inline bool first_use_on_device(bool (&done)[16]) {
+// A launcher's once-per-device set-up (kernel attributes are set per device): runs
+// `setup` the first time any thread asks for the current device; other threads
+// asking meanwhile wait for it.  Returns setup's result to the thread that ran it.
+template <typename Setup>
+inline cudaError_t once_per_device(std::once_flag (&flags)[16], Setup&& setup) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return true;
-    if (done[dev]) return false;
-    done[dev] = true;
-    return true;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return setup();
+    cudaError_t e = cudaSuccess;
+    std::call_once(flags[dev], [&] { e = setup(); });
+    return e;
 }
 
 // ---------------------------------------------------------------- launchers

@@ -188,12 +188,12 @@ bool router_tc_supported(int E, int H, int k, int T) {
 cudaError_t launch_router_tc(const CUtensorMap& xmap, const RouterTcArgs& a, int pdl,
                              cudaStream_t s) {
     if (!router_tc_supported(kE, a.H, a.k, a.T)) return cudaErrorInvalidValue;
-    static bool configured[16] = {};    // per device: the attribute is set per device
-    if (first_use_on_device(configured)) {
-        cudaError_t e = cudaFuncSetAttribute(router_tc_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-        if (e != cudaSuccess) return e;
-    }
+    static std::once_flag configured[16];    // the attribute is set per device
+    cudaError_t e = once_per_device(configured, [] {
+        return cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kSmem);
+    });
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1);
     cfg.blockDim = dim3(kThreads);

@@ -444,15 +444,17 @@ cudaError_t launch_router_t(const RouterArgs& a, dim3 grid, size_t smem, int pdl
     // Every instance may take up to kMaxRouterSmem bytes of dynamic shared memory; the
     // attribute is set once per instance (the three instances share one signature, so
     // a per-call "already allowed" record could not tell them apart).
-    static bool configured[16] = {};    // per device: the attribute is set per device
-    if (first_use_on_device(configured)) {
+    static std::once_flag configured[16];    // the attribute is set per device
+    cudaError_t e = once_per_device(configured, [] {
         for (auto kernel : {router_kernel<Tin, VEC, 4>, router_kernel<Tin, VEC, 8>,
                             router_kernel<Tin, VEC, 32>}) {
-            cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  kMaxRouterSmem);
-            if (e != cudaSuccess) return e;
+            if (r != cudaSuccess) return r;
         }
-    }
+        return cudaSuccess;
+    });
+    if (e != cudaSuccess) return e;
     auto go = [&](auto kernel) -> cudaError_t {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = grid;
