@@ -111,9 +111,9 @@ moe_status moe_route(moe_handle h, const void* x, int T, int32_t* topk_idx,
  * combine, each kernel a programmatic dependent of the one before.  Up to 64
  * tokens with 128 experts and no pre-norm, the router is one CTA that forms the
  * logits on the tensor cores (fp32 accumulate), so its routing can differ from
- * moe_route's CUDA-core logits by fp32 rounding (weights) and at exact near-ties.  Larger calls
- * run router, permutation, one grouped expert GEMM launch (the shared expert's
- * tiles among the routed experts') and combine.
+ * moe_route's CUDA-core logits by fp32 rounding (weights) and at exact
+ * near-ties.  Larger calls run router, permutation, one grouped expert GEMM
+ * launch (the shared expert's tiles among the routed experts') and combine.
  */
 moe_status moe_forward(moe_handle h, const void* x, const void* residual, void* y,
                        int T, int32_t* topk_idx_out, float* topk_w_out, void* stream);
