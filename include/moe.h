@@ -29,6 +29,9 @@
  *    and until then every call that starts after the faulty work has finished
  *    returns it without launching anything.
  *  - The library never takes ownership of caller memory.
+ *  - A handle is not thread-safe: calls on one handle share its workspace and
+ *    must be serialised by the caller (and, across streams, ordered on the GPU).
+ *    Different handles are independent; moe_route_noalloc has its own rule.
  */
 #ifndef SPARSE_MOE_B200_MOE_H
 #define SPARSE_MOE_B200_MOE_H
