@@ -429,6 +429,34 @@ def main():
     kern = {c: {"launches": n, "mean_us": (t / n * 1e3) if n else None}
             for c, (n, t) in per_class.items()}
 
+    # ---- per-call latency: one single-call graph per weight copy, each replay between
+    # two events on the bench stream (device time of one forward call; p50/p95/p99)
+    lat = None
+    if use_graph:
+        one = []
+        for r in range(rotate):
+            g1 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g1, stream=stream):
+                step(r)
+            one.append(g1)
+        n_lat = min(400, max(20, steps_timed))
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n_lat)]
+        with torch.cuda.stream(stream):
+            for i, (e0, e1) in enumerate(evs):
+                e0.record(stream)
+                one[i % rotate].replay()
+                e1.record(stream)
+        torch.cuda.synchronize()
+        us = np.array([e0.elapsed_time(e1) * 1e3 for e0, e1 in evs])
+        lat = {"p50": float(np.percentile(us, 50)), "p95": float(np.percentile(us, 95)),
+               "p99": float(np.percentile(us, 99)), "unit": "us", "calls": n_lat,
+               "what": "device time of one call, single-call CUDA graph between events"}
+        del one
+    for hs in handles:
+        for layer in hs:
+            layer.kernel_stats(reset=True)
+
     # ---- roofline of the dominant kernel (the expert kernel)
     peaks = load_peaks()
     ex_n, ex_ms = per_class.get("experts", (0, 0.0))
@@ -519,7 +547,7 @@ def main():
                 "dtype": wl.dtype, "data": "synthetic (seeded; random-init weights)",
                 "impl": "ours", "config": workload_config(wl, world, rotate, l2),
                 "timing": "CUDA graphs of captured forward calls" if use_graph else "eager",
-                "roofline": roof, "layer": whole, "kernels": kern,
+                "roofline": roof, "layer": whole, "kernels": kern, "latency": lat,
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
                 "clocks": clocks.summary()}
         print(json.dumps(line), flush=True)
