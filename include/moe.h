@@ -48,7 +48,7 @@ typedef enum {
     MOE_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or option      */
     MOE_ERR_CUDA = 2,          /* a CUDA runtime/driver call failed           */
     MOE_ERR_OOM = 3,           /* device or pinned-host allocation failed      */
-    MOE_ERR_UNSUPPORTED = 4,   /* shape/dtype this build has no kernel for     */
+    MOE_ERR_UNSUPPORTED = 4,   /* shape/dtype the library has no kernel for   */
     MOE_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out           */
     MOE_ERR_DEVICE_CHECK = 6   /* a device-side consistency check failed       */
 } moe_status;

@@ -35,10 +35,17 @@ def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
     stale = force or not os.path.exists(out) or any(
         os.path.getmtime(p) > os.path.getmtime(out) for p in (src, _HDR))
     if stale:
+        # a private temporary per process, then an atomic replace: several processes
+        # (e.g. the ranks of a multi-process test) may rebuild at the same time
+        tmp = f"{out}.{os.getpid()}.tmp"
         cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
-               "-I", _HERE, src, "-o", out + ".tmp", "-lm"]
-        subprocess.run(cmd, check=True)
-        os.replace(out + ".tmp", out)
+               "-I", _HERE, src, "-o", tmp, "-lm"]
+        try:
+            subprocess.run(cmd, check=True)
+            os.replace(tmp, out)
+        finally:
+            if os.path.exists(tmp):
+                os.remove(tmp)
     return out
 
 

@@ -1,7 +1,7 @@
 /*
  * moe_oracle.c -- plain, slow, fp64 CPU oracle of one sparse MoE FFN layer.
  *
- * TEST INFRASTRUCTURE ONLY: it judges the CUDA path and is never part of it.
+ * TEST INFRASTRUCTURE ONLY: it checks the CUDA path and is never part of it.
  * Every step below follows the layer's definition literally, one token at a
  * time, with no blocking, fusion or reordering.  The passages each function
  * follows are cited above it; the full statement is in moe_oracle.h.

@@ -1,7 +1,7 @@
 /*
  * moe_oracle.h -- plain fp64 CPU oracle of one sparse MoE feed-forward layer.
  *
- * TEST INFRASTRUCTURE ONLY.  This oracle exists to judge the CUDA path.  Only
+ * TEST INFRASTRUCTURE ONLY.  This oracle exists to check the CUDA path.  Only
  * the test suite, the smoke check and the benchmark's CPU-baseline leg may
  * load it.  It shares no code, header, table or helper with the CUDA library.
  *
