@@ -75,3 +75,34 @@ def test_binding_fails_loudly_without_library(tmp_path):
             smt.load(str(tmp_path / "missing.so"))
         finally:
             smt._lib = smt._lib_backup
+
+
+def test_noalloc_argument_errors_without_gpu(lib):
+    """moe_route_noalloc rejects bad arguments before it touches the CUDA runtime
+    (the pointer values below are never dereferenced)."""
+    P = ctypes.c_void_p
+    ok = smt._Config(1024, 128, 6, 384, 768, smt.DTYPE_BF16, 1, 1e-6)
+    x, w, idx, wt = P(256), P(512), P(1024), P(2048)
+
+    def call(cfg, T, x=x, w=w, idx=idx, wt=wt):
+        return lib.moe_route_noalloc(None if cfg is None else ctypes.byref(cfg), x, w, None, T,
+                                     idx, wt, None)
+
+    assert call(None, 8) == smt.MOE_ERR_INVALID_ARG
+    for bad in (smt._Config(0, 128, 6, 384, 768, smt.DTYPE_BF16, 1, 1e-6),      # H = 0
+                smt._Config(1024, 2048, 6, 384, 768, smt.DTYPE_BF16, 1, 1e-6),  # E > 1024
+                smt._Config(1024, 4, 6, 384, 768, smt.DTYPE_BF16, 1, 1e-6),     # k > E
+                smt._Config(1024, 128, 17, 384, 768, smt.DTYPE_BF16, 1, 1e-6),  # k > 16
+                smt._Config(1024, 128, 6, 384, 768, 7, 1, 1e-6)):               # dtype
+        assert call(bad, 8) == smt.MOE_ERR_INVALID_ARG
+    nr = smt._Config(1024, 128, 6, 384, 768, smt.DTYPE_BF16, 0, 1e-6)
+    assert call(nr, 8) == smt.MOE_ERR_UNSUPPORTED
+    assert call(ok, -1) == smt.MOE_ERR_INVALID_ARG
+    assert call(ok, 0, x=None, w=None, idx=None, wt=None) == smt.MOE_OK       # T = 0: no-op
+    assert call(ok, 8, x=None) == smt.MOE_ERR_INVALID_ARG
+    assert call(ok, 8, idx=None) == smt.MOE_ERR_INVALID_ARG
+    assert call(ok, 8, x=P(264)) == smt.MOE_ERR_INVALID_ARG                    # misaligned
+    assert b"aligned" in lib.moe_last_error(None)
+    # the fixed scratch holds T = 8183 tokens at E = 128; one more is refused
+    assert call(ok, 8184) == smt.MOE_ERR_INVALID_ARG
+    assert b"fixed" in lib.moe_last_error(None)
