@@ -239,8 +239,9 @@ def pin_numpy_statement(make):
 
 def pin_rms_residual_gap(make):
     """R: pre-RMSNorm closed form (x = (3, 4, 0, ...), eps = 0: mean x^2 = 25/H, so the
-    normalised input is (3, 4, 0, ...) * sqrt(H) / 5 times the scale g); the residual is
-    added exactly; the k-gap equals the k-th minus the (k+1)-th sorted logit."""
+    normalised input is (3, 4, 0, ...) * sqrt(H) / 5 times the scale g; and with eps = 1/2
+    at H = 16); the residual is added exactly; the k-gap equals the k-th minus the
+    (k+1)-th sorted logit."""
     rng = np.random.default_rng(8)
     H = 16
     lw = _f64_layer(rng, H, 8, 3, 6, 4)
@@ -254,6 +255,13 @@ def pin_rms_residual_gap(make):
     assert np.array_equal(idx_rms, idx_plain) and _rel(y_rms, y_plain) < 1e-13
     y_raw, *_ = make(lw).forward(x * 7.0)
     assert _rel(y_raw, y_plain) > 1e-3          # the norm matters: the pin is not vacuous
+    # eps sits inside the square root: eps = 1/2 gives mean x^2 + eps = 25/16 + 8/16, so the
+    # normalised input is (3, 4, 0, ...) * 4 / sqrt(33) times g
+    with_eps = LayerWeights(lw.w_router, lw.w_gate, lw.w_up, lw.w_down, lw.ws_gate, lw.ws_up,
+                            lw.ws_down, rms_w=g, rms_eps=0.5, top_k=3)
+    y_eps, idx_eps, *_ = make(with_eps).forward(x)
+    y_ref, idx_ref, *_ = make(lw).forward(x * 4.0 / math.sqrt(33.0) * g)
+    assert np.array_equal(idx_eps, idx_ref) and _rel(y_eps, y_ref) < 1e-13
     x = rng.standard_normal((7, H))
     r = rng.standard_normal((7, H))
     o = make(lw)

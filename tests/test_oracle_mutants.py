@@ -29,6 +29,18 @@ MUTANTS = {
     "residual_dropped": ("y[(size_t)t * H + o] = acc[o] + r;", "y[(size_t)t * H + o] = acc[o];"),
     "softmax_temperature": ("p[e] = exp(l[e] - m);", "p[e] = exp(2.0 * (l[e] - m));"),
     "routed_unweighted": ("acc[o] += ws[i] * eo[o];", "acc[o] += eo[o];"),
+    "rms_eps_outside_sqrt": ("double r = sqrt(ms + c->rms_eps);",
+                             "double r = sqrt(ms) + c->rms_eps;"),
+    "rms_scale_dropped": ("v[j] = v[j] / r * load(w->rms_w, c->dtype, (size_t)j);",
+                          "v[j] = v[j] / r;"),
+    "shared_up_is_gate": ("swiglu(w->ws_gate, w->ws_up, w->ws_down,",
+                          "swiglu(w->ws_gate, w->ws_gate, w->ws_down,"),
+    "kgap_of_probabilities": ("l[order[k - 1]] - l[order[k]]", "p[order[k - 1]] - p[order[k]]"),
+    "every_token_reads_row_0": ("v[j] = load(x, c->dtype, (size_t)t * H + j);",
+                                "v[j] = load(x, c->dtype, (size_t)j);"),
+    "down_rows_by_inter": ("e * I, e * H, H, I", "e * I, e * I, H, I"),
+    "one_expert_short": ("for (int i = 0; i < k; ++i) psum += p[sel[i]];",
+                         "for (int i = 0; i < k - 1; ++i) psum += p[sel[i]];"),
 }
 
 
