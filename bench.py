@@ -192,9 +192,10 @@ def build_inputs(name, rank, rotate):
     return wl, copies
 
 
-def algorithmic_work(wl, idx_list):
+def algorithmic_work(wl, idx_list, residual=False):
     """Per-step algorithmic bytes / FLOPs of the whole layer and of the routed-expert
-    kernel, from the realised routing (weights of experts with >= 1 token)."""
+    kernel, from the realised routing (weights of experts with >= 1 token); a residual
+    input adds its T x H read."""
     H, E, k, I, Is = wl.H, wl.E, wl.k, wl.I, wl.Is
     es = 2 if wl.dtype == "bf16" else 4
     out = []
@@ -202,7 +203,9 @@ def algorithmic_work(wl, idx_list):
         T = idx.shape[0]
         touched = int(np.unique(idx).size)
         experts_bytes = touched * 3 * H * I * es + 2 * T * k * H * es
-        layer_bytes = es * (H * E + touched * 3 * H * I + 3 * H * Is + 2 * T * H) + T * k * 8
+        act_rows = 3 if residual else 2          # x, y (and the residual)
+        layer_bytes = (es * (H * E + touched * 3 * H * I + 3 * H * Is + act_rows * T * H)
+                       + T * k * 8)
         experts_flops = 2 * 3 * H * I * T * k
         layer_flops = T * (2 * H * E + k * 2 * 3 * H * I + 2 * 3 * H * Is)
         out.append(dict(touched=touched, experts_bytes=experts_bytes, layer_bytes=layer_bytes,
@@ -338,7 +341,7 @@ def main():
                 idx_list.append(idx.cpu().numpy())
                 h = y
     torch.cuda.synchronize()
-    work = algorithmic_work(wl, idx_list)
+    work = algorithmic_work(wl, idx_list, residual=stack)
     for hs in handles:
         for layer in hs:
             st = layer.check(stream)

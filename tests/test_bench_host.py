@@ -50,6 +50,9 @@ def test_algorithmic_work_counts_moved_arrays_and_products():
         assert w["layer_bytes"] == (L.w_router.nbytes + expert_w + L.ws_gate.nbytes
                                     + L.ws_up.nbytes + L.ws_down.nbytes
                                     + 2 * inp.x.nbytes + topk)
+        (wr,) = bench.algorithmic_work(wl, [idx], residual=True)
+        assert wr["layer_bytes"] == w["layer_bytes"] + inp.x.nbytes   # the residual's read
+        assert all(wr[key] == w[key] for key in w if key != "layer_bytes")
         mm = lambda m, n, p: 2 * m * n * p                 # FLOPs of an (m,n)x(n,p) product
         per_slot = mm(1, H, I) + mm(1, H, I) + mm(1, I, H)
         assert w["experts_flops"] == T * k * per_slot
