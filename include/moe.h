@@ -211,7 +211,12 @@ moe_status moe_destroy(moe_handle h);
  * the array: calls whose work overlaps on the GPU (different streams, or other
  * threads) race and must be serialised by the caller.  Logits are always
  * formed on CUDA cores (fp32), so for T >= 256 results can differ from
- * moe_route's tensor-core logits by rounding (near-tie tokens only).
+ * moe_route's tensor-core logits by rounding (near-tie tokens only).  The
+ * router has no device-side wait; its one device check (a selected index out
+ * of range, impossible for 1 <= k <= E) is not reported by this entry point,
+ * which has no handle for moe_check.  Errors: INVALID_ARG (NULL cfg or
+ * pointer, bad sizes or dtype, misaligned x, T too large), UNSUPPORTED
+ * (norm_topk_prob != 1), CUDA (no current device, launch failure).
  */
 moe_status moe_route_noalloc(const moe_config* cfg, const void* x, const void* w_router,
                              const void* rms_weight, int T, int32_t* topk_idx, float* topk_w,
