@@ -11,7 +11,7 @@ weights from being served out of the 126 MB L2, decode steps cycle through 8
 independent weight copies (2.46 GB); prefill steps touch >300 MB each anyway.
 
 The timed loop replays CUDA graphs of captured forward calls (the same kernels a
-forward launches; graphs remove per-call host overhead).  With N > 1 (torchrun)
+forward launches; graphs remove per-call host overhead), exactly --steps of them.  With N > 1 (torchrun)
 every rank runs its own replica on its own tokens (weak scaling, no collective
 on the data path); the time is the max over ranks.
 
@@ -213,6 +213,17 @@ def algorithmic_work(wl, idx_list, residual=False):
     return out
 
 
+def graph_plan(K, rotate, per_graph=32):
+    """How CUDA graphs time exactly K steps: a graph of `cycle` steps (whole rotation
+    cycles of the weight copies when K allows; step i uses copy i % rotate) replayed
+    n_rep times, then a graph of the remaining `rem` steps (starting again at copy 0)."""
+    if K < 1:
+        raise ValueError("--steps must be >= 1")
+    cycle = min(K, rotate * max(1, per_graph // rotate))
+    n_rep, rem = divmod(K, cycle)
+    return cycle, n_rep, rem
+
+
 # ----------------------------------------------------------------------------- CPU arms
 def oracle_sample_rate(wl, layers, x, seconds):
     """Tokens/s of the fp64 oracle on this host's cores over a bounded sample."""
@@ -347,14 +358,14 @@ def main():
             st = layer.check(stream)
             assert st == 0, f"device-side status {st}"
 
-    # ---- warm-up, then CUDA graphs covering whole rotation cycles
+    # ---- warm-up, then CUDA graphs that together hold exactly K steps
     for i in range(W):
         with torch.cuda.stream(stream):
             step(i % rotate)
     torch.cuda.synchronize()
     use_graph = not args.no_graph
-    cycle = rotate * max(1, 32 // rotate) if use_graph else rotate
-    graph = None
+    cycle, n_rep, rem = graph_plan(K, rotate)
+    graph = graph_rem = None
     launches_per_step = 0.0
     if use_graph:
         for hs in handles:
@@ -367,11 +378,17 @@ def main():
         # every launch the library made while capturing is a kernel node of the graph
         launches_per_step = sum(n for hs in handles for layer in hs
                                 for n, _ in layer.kernel_stats(reset=True).values()) / cycle
+        if rem:
+            graph_rem = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph_rem, stream=stream):
+                for i in range(rem):
+                    step(i % rotate)
         with torch.cuda.stream(stream):
             graph.replay()
+            if graph_rem is not None:
+                graph_rem.replay()
         torch.cuda.synchronize()
-    n_rep = max(1, -(-K // cycle)) if use_graph else K
-    steps_timed = n_rep * cycle if use_graph else K
+    steps_timed = K
     for hs in handles:
         for layer in hs:
             layer.kernel_stats(reset=True)
@@ -388,6 +405,8 @@ def main():
             with torch.cuda.stream(stream):      # replay on the stream the events time
                 for _ in range(n_rep):
                     graph.replay()
+                if graph_rem is not None:
+                    graph_rem.replay()
         else:
             with torch.cuda.stream(stream):
                 for i in range(K):
@@ -538,8 +557,7 @@ def main():
     for hs in handles:
         for layer in hs:
             assert layer.check(stream) == 0
-    if graph is not None:
-        del graph
+    del graph, graph_rem
     if rank == 0:
         l2 = (f"rotate {rotate} independent weight copies ({rotate * copies[0][0][0].nbytes / 1e9:.2f}"
               f" GB) > 126 MB L2" if rotate > 1 else

@@ -151,3 +151,22 @@ def test_reference_arm_other_ranks_are_silent():
     r = _run_reference({"RANK": "1", "LOCAL_RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_graph_plan_times_exactly_k_steps():
+    """The captured graphs hold exactly K timed steps, and with several weight copies
+    no two consecutive steps read the same copy (each step misses in L2)."""
+    import pytest
+    for rotate in (1, 3, 8):
+        for K in list(range(1, 80)) + [400, 20000, 20001]:
+            cycle, n_rep, rem = bench.graph_plan(K, rotate)
+            assert cycle * n_rep + rem == K and 1 <= cycle <= 32 and 0 <= rem < cycle
+            if K >= 32:
+                assert cycle % rotate == 0          # replays start again at copy 0
+            copies = [i % rotate for i in range(cycle)] * n_rep + [i % rotate
+                                                                   for i in range(rem)]
+            assert len(copies) == K
+            if rotate > 1:
+                assert all(a != b for a, b in zip(copies, copies[1:]))
+    with pytest.raises(ValueError):
+        bench.graph_plan(0, 8)
