@@ -21,8 +21,10 @@ Reported besides the device throughput:
   roofline      routed-expert kernel: algorithmic bytes (touched expert weights +
                 its input and output rows) or FLOPs per launch / its mean
                 CUDA-event duration, against MEASURED_PEAKS.json
-  cpu_baseline  the fp64 oracle on this host's cores over a bounded sample
+  cpu_baseline  the fp64 oracle on this host's cores over a bounded sample (and on
+                one thread over half that time), with the CPU model
   clocks        nvidia-smi samples taken during the timed loop
+  env           GPU name, driver, CUDA runtime, torch and library versions
 --impl reference times the oracle alone (the CPU reference arm).
 """
 from __future__ import annotations
@@ -166,6 +168,24 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def run_env(torch, dev, smt, gpu_uuid):
+    """Run conditions: GPU name, driver, CUDA runtime, torch and library versions
+    (None for anything that cannot be read)."""
+    def driver():
+        r = subprocess.run(["nvidia-smi", "-i", gpu_uuid, "--query-gpu=driver_version",
+                            "--format=csv,noheader"], capture_output=True, text=True, timeout=20)
+        return r.stdout.strip() or None
+    env = {}
+    for key, fn in (("gpu", lambda: torch.cuda.get_device_name(dev)), ("driver", driver),
+                    ("cuda_runtime", lambda: torch.version.cuda),
+                    ("torch", lambda: torch.__version__), ("library", lambda: smt.version())):
+        try:
+            env[key] = fn()
+        except Exception:
+            env[key] = None
+    return env
+
+
 def max_over_ranks(value: float, dist=None, device=None) -> float:
     """Largest value across ranks (the timing rule: the slowest rank sets the time)."""
     if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
@@ -225,10 +245,23 @@ def graph_plan(K, rotate, per_graph=32):
 
 
 # ----------------------------------------------------------------------------- CPU arms
-def oracle_sample_rate(wl, layers, x, seconds):
-    """Tokens/s of the fp64 oracle on this host's cores over a bounded sample."""
+def cpu_model():
+    """The host CPU's model name (Linux), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def oracle_sample_rate(wl, layers, x, seconds, nthreads=None):
+    """Tokens/s of the fp64 oracle on this host's cores (or on `nthreads` threads) over
+    a bounded sample (whole token batches until `seconds` have passed)."""
     import oracle
-    cores = len(os.sched_getaffinity(0))
+    cores = nthreads or len(os.sched_getaffinity(0))
     T = x.shape[0]
     n_tok = T if wl.n_layers > 1 or T <= 64 else 64
     xs = x[:n_tok]
@@ -551,8 +584,11 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
         v, threads, sample = oracle_sample_rate(wl, copies[0][0], copies[0][1], args.cpu_seconds)
+        v1, _, sample1 = oracle_sample_rate(wl, copies[0][0], copies[0][1],
+                                            args.cpu_seconds / 2, nthreads=1)
         cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": sample}
+               "sample": sample, "cpu_model": cpu_model(),
+               "single_thread": {"value": v1, "unit": "tokens/s", "sample": sample1}}
 
     for hs in handles:
         for layer in hs:
@@ -570,7 +606,7 @@ def main():
                 "timing": "CUDA graphs of captured forward calls" if use_graph else "eager",
                 "roofline": roof, "layer": whole, "kernels": kern, "latency": lat,
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-                "clocks": clocks.summary()}
+                "clocks": clocks.summary(), "env": run_env(torch, dev, smt, gpu_uuid)}
         print(json.dumps(line), flush=True)
     for hs in handles:
         for layer in hs:
