@@ -1,5 +1,5 @@
 // topk.cuh -- warp Top-k selection with renormalised weights, shared by the
-// router kernels and the few-token expert kernel (which routes for itself).
+// CUDA-core router (routing.cu) and the one-CTA tensor-core router (router_tc.cu).
 //
 // Router equation: page "3C . Talker MoE (20 lop, 128 Experts Top-6) & Dau ra
 // ma ngu nghia c_0", section 3: p = softmax(W_r x), S = Top-k, w_i = p_i /
