@@ -170,3 +170,22 @@ def test_graph_plan_times_exactly_k_steps():
                 assert all(a != b for a, b in zip(copies, copies[1:]))
     with pytest.raises(ValueError):
         bench.graph_plan(0, 8)
+
+
+def test_reference_arm_under_torchrun():
+    """Launched like the multi-GPU bench (torchrun, two ranks): one line, from rank 0."""
+    import socket
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        port = sock.getsockname()[1]
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                        "--nproc-per-node", "2", "--master-addr", "127.0.0.1",
+                        "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+                        "--impl", "reference", "--workload", "tiny_fp32", "--gpus", "2",
+                        "--steps", "3", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["steps"] == 3
