@@ -11,11 +11,14 @@ deliberately broken copy of the C oracle) and raises AssertionError on failure.
   O6  special cases: E=1,k=1 dense MLPs; k=E softmax mixture; identical experts;
       zero router (all ties -> lower indices, w = 1/k)
   O7  independent NumPy statement agrees with the C oracle
+  O8  bf16 storage at the Talker size: bf16 bits == their exact fp64 values, bit for
+      bit, and == a brute-force dense evaluation of all 128 experts on a token sample
   R   pre-RMSNorm and residual special cases; k-gap equals the sorted-logit gap
 """
 from __future__ import annotations
 
 import ast
+import functools
 import math
 import operator
 import os
@@ -274,6 +277,46 @@ def pin_rms_residual_gap(make):
     assert np.max(np.abs(logits - x @ lw.w_router.T)) < 1e-12
 
 
+@functools.lru_cache(maxsize=1)
+def _talker_sample():
+    """Talker decode weights (bf16 bits and their exact fp64 values), three of its tokens,
+    and the brute-force dense evaluation of all E experts on them (numpy fp64, once)."""
+    inp = synth.make("talker_decode")
+    L = inp.layers[0]
+    W = {n: numpy_ref.widen(a) for n, a in L.arrays().items()}
+    rows = [0, 3, 7]
+    x = numpy_ref.widen(inp.x[rows])
+    k = inp.workload.k
+    logits = x @ W["w_router"].T
+    p = np.exp(logits - logits.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    g = np.einsum("eih,th->tei", W["w_gate"], x)
+    u = np.einsum("eih,th->tei", W["w_up"], x)
+    every = np.einsum("ehi,tei->teh", W["w_down"], _silu(g) * u)     # [T, E, H]: all experts
+    S = np.array([sorted(range(p.shape[1]), key=lambda e: (-logits[t, e], e))[:k]
+                  for t in range(len(rows))], dtype=np.int32)
+    mask = np.zeros_like(p)
+    np.put_along_axis(mask, S, 1.0, axis=1)
+    wts = mask * p / (mask * p).sum(1, keepdims=True)
+    y = np.einsum("te,teh->th", wts, every) + _dense_swiglu(x, W["ws_gate"], W["ws_up"],
+                                                            W["ws_down"])
+    return inp, L, W, rows, x, S, y
+
+
+def pin_bf16_talker_size(make):
+    """O8: at H=1024, E=128, k=6, I=384, I_s=768 with bf16 storage, the oracle on the bit
+    patterns equals the oracle on their exact fp64 values bit for bit (bf16 is the upper
+    half of a binary32), and both match the brute-force dense evaluation within 1e-12."""
+    inp, L, W, rows, x, S, y_ref = _talker_sample()
+    k = inp.workload.k
+    y_bf, idx_bf, w_bf, _ = make(LayerWeights(**L.arrays(), top_k=k)).forward(inp.x[rows])
+    y_64, idx_64, w_64, _ = make(LayerWeights(**W, top_k=k)).forward(x)
+    assert np.array_equal(idx_bf, idx_64) and np.array_equal(y_bf, y_64)
+    assert np.array_equal(w_bf, w_64)
+    assert np.array_equal(idx_bf, S)
+    assert _rel(y_bf, y_ref) < 1e-12
+
+
 ALL_PINS = [pin_weights_sum_to_one, pin_brute_force_dense, pin_expert_permutation,
             pin_token_independence, pin_hand_case, pin_special_cases, pin_numpy_statement,
-            pin_rms_residual_gap]
+            pin_rms_residual_gap, pin_bf16_talker_size]

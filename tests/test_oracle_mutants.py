@@ -39,6 +39,8 @@ MUTANTS = {
     "every_token_reads_row_0": ("v[j] = load(x, c->dtype, (size_t)t * H + j);",
                                 "v[j] = load(x, c->dtype, (size_t)j);"),
     "down_rows_by_inter": ("e * I, e * H, H, I", "e * I, e * I, H, I"),
+    "bf16_decoded_one_bit_low": ("uint32_t bits = (uint32_t)((const uint16_t*)p)[i] << 16;",
+                                 "uint32_t bits = (uint32_t)((const uint16_t*)p)[i] << 15;"),
     "one_expert_short": ("for (int i = 0; i < k; ++i) psum += p[sel[i]];",
                          "for (int i = 0; i < k - 1; ++i) psum += p[sel[i]];"),
 }
