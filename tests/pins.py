@@ -13,6 +13,8 @@ deliberately broken copy of the C oracle) and raises AssertionError on failure.
   O7  independent NumPy statement agrees with the C oracle
   O8  bf16 storage at the Talker size: bf16 bits == their exact fp64 values, bit for
       bit, and == a brute-force dense evaluation of all 128 experts on a token sample
+  O9  forced routing (the near-tie re-evaluation): forcing the oracle's own sets changes
+      nothing; forcing other sets gives the masked dense evaluation over those sets
   R   pre-RMSNorm and residual special cases; k-gap equals the sorted-logit gap
 """
 from __future__ import annotations
@@ -317,6 +319,34 @@ def pin_bf16_talker_size(make):
     assert _rel(y_bf, y_ref) < 1e-12
 
 
+def pin_forced_routing(make):
+    """O9: forward(x, forced_idx=S') uses the sets S' as given: forcing the oracle's own
+    selection is the identity (bit for bit), and any other set gives the dense evaluation
+    of every expert masked to S', weights p_i / sum_{j in S'} p_j, indices in S' order."""
+    rng = np.random.default_rng(9)
+    H, E, k = 10, 7, 3
+    lw = _f64_layer(rng, H, E, k, 6, 5)
+    x = rng.standard_normal((6, H))
+    o = make(lw)
+    y, idx, w, _ = o.forward(x)
+    y2, idx2, w2, _ = o.forward(x, forced_idx=idx)
+    assert np.array_equal(y2, y) and np.array_equal(idx2, idx) and np.array_equal(w2, w)
+    forced = np.array([rng.permutation(E)[:k] for _ in range(x.shape[0])], dtype=np.int32)
+    y3, idx3, w3, _ = o.forward(x, forced_idx=forced)
+    assert np.array_equal(idx3, forced)
+    logits = x @ lw.w_router.T
+    p = np.exp(logits - logits.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    every = np.stack([_dense_swiglu(x, lw.w_gate[e], lw.w_up[e], lw.w_down[e])
+                      for e in range(E)], axis=1)
+    mask = np.zeros_like(p)
+    np.put_along_axis(mask, forced, 1.0, axis=1)
+    wts = mask * p / (mask * p).sum(1, keepdims=True)
+    ref = np.einsum("te,teh->th", wts, every) + _dense_swiglu(x, lw.ws_gate, lw.ws_up, lw.ws_down)
+    assert _rel(y3, ref) < 1e-12
+    assert np.max(np.abs(w3 - np.take_along_axis(wts, forced, axis=1))) < 1e-15
+
+
 ALL_PINS = [pin_weights_sum_to_one, pin_brute_force_dense, pin_expert_permutation,
             pin_token_independence, pin_hand_case, pin_special_cases, pin_numpy_statement,
-            pin_rms_residual_gap, pin_bf16_talker_size]
+            pin_rms_residual_gap, pin_bf16_talker_size, pin_forced_routing]

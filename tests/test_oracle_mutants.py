@@ -41,6 +41,8 @@ MUTANTS = {
     "down_rows_by_inter": ("e * I, e * H, H, I", "e * I, e * I, H, I"),
     "bf16_decoded_one_bit_low": ("uint32_t bits = (uint32_t)((const uint16_t*)p)[i] << 16;",
                                  "uint32_t bits = (uint32_t)((const uint16_t*)p)[i] << 15;"),
+    "forced_sets_ignored": ("sel[i] = forced ? forced[i] : order[i];", "sel[i] = order[i];"),
+    "forced_weights_from_own_sets": ("psum += p[sel[i]];", "psum += p[order[i]];"),
     "one_expert_short": ("for (int i = 0; i < k; ++i) psum += p[sel[i]];",
                          "for (int i = 0; i < k - 1; ++i) psum += p[sel[i]];"),
 }
