@@ -88,7 +88,11 @@ moe_status moe_create(const moe_config* cfg, int device,
 /*
  * Reserve the device workspace for up to `max_tokens` tokens per call.  Calls
  * with T <= max_tokens then allocate nothing, which is what makes a forward
- * capturable in a CUDA graph.  Synchronous.  Errors: INVALID_ARG, OOM, CUDA.
+ * capturable in a CUDA graph.  Synchronous.  The kernels index rows with 32-bit
+ * integers, so max_tokens * (k + 1) * max(H, I, I_s) must stay below 2^31 (at the
+ * Talker sizes: up to 299,593 tokens per call); larger reservations return
+ * UNSUPPORTED and the caller splits the batch.  Errors: INVALID_ARG, UNSUPPORTED,
+ * OOM, CUDA.
  */
 moe_status moe_reserve(moe_handle h, int max_tokens);
 

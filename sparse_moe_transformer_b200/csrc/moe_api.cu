@@ -340,6 +340,13 @@ moe_status moe_create(const moe_config* cfg, int device, const void* w_router, c
 moe_status moe_reserve(moe_handle h, int max_tokens) {
     if (!h || max_tokens < 0) return fail(MOE_ERR_INVALID_ARG, "bad handle or max_tokens");
     if (max_tokens <= h->max_T) return MOE_OK;
+    // The kernels index the per-row buffers (T k + T rows of up to max(H, I, I_s)
+    // elements) with 32-bit integers.
+    const uint64_t width = std::max({(uint64_t)h->d.H, (uint64_t)h->d.I, (uint64_t)h->d.Is});
+    if ((uint64_t)max_tokens * (uint64_t)(h->d.k + 1) * width >= (1ull << 31))
+        return fail(MOE_ERR_UNSUPPORTED,
+                    "max_tokens=%d: T*(k+1)*max(H, I, I_s) must stay below 2^31 "
+                    "(32-bit row indexing); split the batch", max_tokens);
     DeviceGuard g(h->device);
     CUDA_TRY(cudaDeviceSynchronize());
     free_workspace(h);

@@ -281,6 +281,19 @@ def test_zero_tokens_and_growth():
     assert_parity(compare(orc, inp.x, ys, idx, w, "bf16"), "bf16")
 
 
+def test_reserve_refuses_past_32bit_row_indexing():
+    """A reservation with T (k + 1) max(H, I, I_s) >= 2^31 is refused before anything
+    is allocated, and the handle stays usable."""
+    inp = synth.make_custom(256, 16, 4, 128, 128, 40, "bf16", seed=12)
+    layer, orc = _layer(inp)
+    limit = (2**31 - 1) // ((4 + 1) * 256)        # largest T that stays below 2^31
+    with pytest.raises(smt.MoEError) as err:
+        layer.reserve(limit + 1)
+    assert err.value.status == smt.MOE_ERR_UNSUPPORTED
+    ys, idx, w = _run(layer, inp.x)
+    assert_parity(compare(orc, inp.x, ys, idx, w, "bf16"), "bf16")
+
+
 def test_bounded_wait_reports_timeout_and_recovers():
     inp = synth.make_custom(256, 16, 4, 128, 128, 64, "bf16", seed=13)
     layer, orc = _layer(inp)
