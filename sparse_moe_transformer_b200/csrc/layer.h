@@ -206,7 +206,8 @@ struct FusedArgs {
     const int32_t* topk_idx;   // [T][k] from the router
     float* o_part;             // [max(I, Is) / 128][T*k + T][H] fp32
     int H, I, Is, E, k, T;
-    int x_early;               // 1: x_rows exists before the router runs (no pre-norm)
+    int x_early;               // 1: x_rows may be read before the grid dependency wait
+                               // (only safe when nothing in flight writes it)
     const int32_t* zero_word;  // a word that stays 0 (bounded-wait test hook)
     DeviceStatus st;
     uint64_t wait_limit_ns;

@@ -493,7 +493,12 @@ moe_status run_layer_fused(moe_layer* h, const void* x, const void* residual, vo
         FusedArgs a{};
         a.w_gu = h->w_gate; a.w_down = h->w_down;
         a.ws_gu = d.Is ? h->ws_gate : nullptr; a.ws_down = d.Is ? h->ws_down : nullptr;
-        a.x_rows = x_in; a.x_early = h->rms_w ? 0 : 1;
+        // x_early = 0: every CTA waits for the router before reading x.  The router
+        // lets this kernel launch before its own wait on the previous kernel, and the
+        // previous call's combine lets the router launch before it writes y, so when a
+        // call's x is the previous call's y (a residual stream, in place or not) only
+        // the dependency wait orders the read of x after that write.
+        a.x_rows = x_in; a.x_early = 0;
         a.topk_idx = rb.topk_idx; a.o_part = h->o_part;
         a.H = d.H; a.I = d.I; a.Is = d.Is; a.E = d.E; a.k = d.k; a.T = T;
         a.zero_word = h->sync_fused + 2;

@@ -294,6 +294,27 @@ def test_reserve_refuses_past_32bit_row_indexing():
     assert_parity(compare(orc, inp.x, ys, idx, w, "bf16"), "bf16")
 
 
+@pytest.mark.parametrize("T", [8, 64])
+def test_back_to_back_residual_stream(T):
+    """Calls whose input is the previous call's output (an in-place residual stream with
+    no pre-norm, the few-token path with the one-CTA router) give the same bits when
+    issued back to back on one stream as with a device synchronisation after every call:
+    each call reads x only after the previous call has written it."""
+    inp = synth.make("talker_decode", T=T)
+    layer, _ = _layer(inp)
+    x0 = smt.to_device(inp.x)
+    a, b = x0.clone(), x0.clone()
+    for _ in range(48):
+        layer.forward(a, residual=a, out=a)
+    torch.cuda.synchronize()
+    for _ in range(48):
+        layer.forward(b, residual=b, out=b)
+        torch.cuda.synchronize()
+    assert layer.check() == 0
+    assert torch.isfinite(a.float()).all()
+    assert torch.equal(a, b)
+
+
 def test_bounded_wait_reports_timeout_and_recovers():
     inp = synth.make_custom(256, 16, 4, 128, 128, 64, "bf16", seed=13)
     layer, orc = _layer(inp)
