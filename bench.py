@@ -79,13 +79,20 @@ def dist_env():
     return world, rank, local
 
 
-def load_peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
+def load_peaks(path=None):
+    """Measured HBM copy bandwidth and bf16 GEMM throughput of this GPU model, else the
+    fallback figures (an unreadable or incomplete file counts as absent)."""
+    p = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
         with open(p) as f:
             d = json.load(f)
-        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
-                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+        hbm, tf = float(d["hbm_gbs"]), float(d["bf16_tflops"])
+        if hbm > 0 and tf > 0:
+            return {"hbm_gbs": hbm, "bf16_tflops": tf,
+                    "bf16_tflops_sustained": d.get("bf16_tflops_sustained"),
+                    "source": "measured"}
+    except (OSError, ValueError, KeyError, TypeError):
+        pass
     return dict(FALLBACK_PEAKS)
 
 

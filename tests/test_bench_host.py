@@ -189,3 +189,17 @@ def test_reference_arm_under_torchrun():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["steps"] == 3
+
+
+def test_load_peaks(tmp_path):
+    good = tmp_path / "good.json"
+    good.write_text(json.dumps({"hbm_gbs": 6458.1, "bf16_tflops": 1672.0,
+                                "bf16_tflops_sustained": 1408.4}))
+    p = bench.load_peaks(str(good))
+    assert p["source"] == "measured" and p["hbm_gbs"] == 6458.1 and p["bf16_tflops"] == 1672.0
+    for bad in ("{}", "not json", json.dumps({"hbm_gbs": 0, "bf16_tflops": 1.0}),
+                json.dumps({"hbm_gbs": None, "bf16_tflops": 1.0})):
+        f = tmp_path / "bad.json"
+        f.write_text(bad)
+        assert bench.load_peaks(str(f)) == bench.FALLBACK_PEAKS
+    assert bench.load_peaks(str(tmp_path / "missing.json")) == bench.FALLBACK_PEAKS
