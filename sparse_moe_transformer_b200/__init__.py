@@ -152,8 +152,22 @@ class MoELayer:
         if T > self.reserved:
             self.reserve(T)
 
+    def _check_tokens(self, x, **others):
+        """x: a contiguous [T, hidden] tensor of the layer dtype on a CUDA device; each
+        other tensor (residual, out) either None or of exactly x's shape, dtype, device
+        and layout (the library reads and writes T x hidden elements through them)."""
+        if not (x.is_cuda and x.is_contiguous() and x.dtype == self.torch_dtype and
+                x.dim() == 2 and x.shape[1] == self.cfg.hidden):
+            raise ValueError(f"x must be a contiguous [T, {self.cfg.hidden}] "
+                             f"{self.torch_dtype} CUDA tensor")
+        for name, t in others.items():
+            if t is not None and not (t.shape == x.shape and t.dtype == x.dtype and
+                                      t.device == x.device and t.is_contiguous()):
+                raise ValueError(f"{name} must match x (shape, dtype, device, contiguous)")
+
     def route(self, x, stream=None):
         import torch
+        self._check_tokens(x)
         T = x.shape[0]
         self._ensure(T)
         idx = torch.empty((T, self.cfg.top_k), dtype=torch.int32, device=x.device)
@@ -164,9 +178,9 @@ class MoELayer:
 
     def forward(self, x, residual=None, out=None, return_routing=False, stream=None):
         import torch
+        self._check_tokens(x, residual=residual, out=out)
         T = x.shape[0]
         self._ensure(T)
-        assert x.is_contiguous() and x.dtype == self.torch_dtype
         y = torch.empty_like(x) if out is None else out
         idx = w = None
         if return_routing:
@@ -178,6 +192,13 @@ class MoELayer:
 
     def forward_host(self, x_host, y_host, residual_host=None, stream=None):
         """x_host / y_host: (pinned) CPU tensors [T, H]; synchronous."""
+        for name, t in (("x_host", x_host), ("y_host", y_host), ("residual_host", residual_host)):
+            if t is not None and not (not t.is_cuda and t.is_contiguous() and
+                                      t.dtype == self.torch_dtype and t.dim() == 2 and
+                                      t.shape == x_host.shape and
+                                      t.shape[1] == self.cfg.hidden):
+                raise ValueError(f"{name} must be a contiguous [T, {self.cfg.hidden}] "
+                                 f"{self.torch_dtype} host tensor shaped like x_host")
         T = x_host.shape[0]
         self._ensure(T)
         _check(self.lib.moe_forward_host(self.handle, _ptr(x_host), _ptr(residual_host),

@@ -106,3 +106,57 @@ def test_noalloc_argument_errors_without_gpu(lib):
     # the fixed scratch holds T = 8183 tokens at E = 128; one more is refused
     assert call(ok, 8184) == smt.MOE_ERR_INVALID_ARG
     assert b"fixed" in lib.moe_last_error(None)
+
+
+class _FakeCudaTensor:
+    """Just enough of a CUDA tensor for the binding's argument checks (no GPU here)."""
+
+    def __init__(self, shape, dtype, contiguous=True, device="cuda:0"):
+        import torch
+        self.shape = torch.Size(shape)
+        self.dtype = dtype
+        self.is_cuda = True
+        self.device = torch.device(device)
+        self._contiguous = contiguous
+
+    def is_contiguous(self):
+        return self._contiguous
+
+    def dim(self):
+        return len(self.shape)
+
+
+def test_binding_argument_checks_without_gpu():
+    """The binding refuses tensors the library would read or write out of bounds, before
+    it calls the library (a bare layer object: no handle is needed to get that far)."""
+    import torch
+    layer = object.__new__(smt.MoELayer)
+    layer.cfg = smt.LayerConfig(64, 8, 2, 128, 128, "bf16")
+    layer.torch_dtype = torch.bfloat16
+    bf = torch.bfloat16
+    x = _FakeCudaTensor((5, 64), bf)
+    layer._check_tokens(x, residual=_FakeCudaTensor((5, 64), bf), out=None)
+    bad_x = [torch.zeros(5, 64, dtype=bf),                        # host tensor
+             _FakeCudaTensor((5, 32), bf),                         # wrong hidden size
+             _FakeCudaTensor((5, 64), torch.float32),              # wrong dtype
+             _FakeCudaTensor((5, 64), bf, contiguous=False),
+             _FakeCudaTensor((5, 2, 32), bf)]
+    for t in bad_x:
+        with pytest.raises(ValueError):
+            layer._check_tokens(t)
+        with pytest.raises(ValueError):
+            layer.forward(t)
+    bad_other = [_FakeCudaTensor((4, 64), bf), _FakeCudaTensor((5, 64), torch.float32),
+                 _FakeCudaTensor((5, 64), bf, contiguous=False),
+                 _FakeCudaTensor((5, 64), bf, device="cuda:1")]
+    for t in bad_other:
+        for name in ("residual", "out"):
+            with pytest.raises(ValueError, match=name):
+                layer._check_tokens(x, **{name: t})
+    xh = torch.zeros(5, 64, dtype=bf)
+    for bad in (torch.zeros(4, 64, dtype=bf), torch.zeros(5, 64, dtype=torch.float32),
+                torch.zeros(64, 5, dtype=bf).t()):
+        with pytest.raises(ValueError):
+            layer.forward_host(xh, bad)
+        with pytest.raises(ValueError):
+            layer.forward_host(xh, torch.zeros(5, 64, dtype=bf), residual_host=bad)
