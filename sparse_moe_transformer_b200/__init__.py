@@ -4,7 +4,7 @@ Argument marshalling only: every step of the layer runs in the CUDA library
 behind include/moe.h.  PyTorch supplies device memory and streams.  There is no
 fallback: if the compiled library is missing this module raises at load time.
 
-    layer = MoELayer.from_tensors(cfg, weights)       # weights: torch CUDA tensors
+    layer = MoELayer(cfg, w_router, w_gate, w_up, w_down, ws_gate, ws_up, ws_down)
     y = layer.forward(x)                              # x: [T, H] CUDA tensor
 """
 from __future__ import annotations
@@ -120,9 +120,20 @@ class MoELayer:
         self.cfg = cfg
         self.device = w_router.device.index if device is None else device
         self.torch_dtype = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
-        for t in (w_router, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, rms_weight):
-            if t is not None:
-                assert t.is_cuda and t.is_contiguous() and t.dtype == self.torch_dtype
+        H, E, I, Is = cfg.hidden, cfg.n_experts, cfg.expert_inter, cfg.shared_inter
+        want = {"w_router": (w_router, (E, H)), "w_gate": (w_gate, (E, I, H)),
+                "w_up": (w_up, (E, I, H)), "w_down": (w_down, (E, H, I)),
+                "ws_gate": (ws_gate, (Is, H)), "ws_up": (ws_up, (Is, H)),
+                "ws_down": (ws_down, (H, Is)), "rms_weight": (rms_weight, (H,))}
+        for name, (t, shape) in want.items():
+            if t is None:
+                if name.startswith("w_") or (name.startswith("ws_") and Is > 0):
+                    raise ValueError(f"{name} is required")
+                continue
+            if not (t.is_cuda and t.is_contiguous() and t.dtype == self.torch_dtype and
+                    tuple(t.shape) == shape):
+                raise ValueError(f"{name} must be a contiguous {list(shape)} "
+                                 f"{self.torch_dtype} CUDA tensor")
         c = _Config(cfg.hidden, cfg.n_experts, cfg.top_k, cfg.expert_inter, cfg.shared_inter,
                     DTYPE_BF16 if cfg.dtype == "bf16" else DTYPE_F32, 1, cfg.rms_eps)
         h = ctypes.c_void_p()

@@ -160,3 +160,32 @@ def test_binding_argument_checks_without_gpu():
             layer.forward_host(xh, bad)
         with pytest.raises(ValueError):
             layer.forward_host(xh, torch.zeros(5, 64, dtype=bf), residual_host=bad)
+
+
+def test_binding_weight_checks_without_gpu():
+    """moe_create copies E x I x H elements and so on from the weight pointers: the
+    binding refuses weights of another shape, dtype or layout before calling it."""
+    import torch
+    bf = torch.bfloat16
+    H, E, k, I, Is = 64, 8, 2, 128, 32
+    cfg = smt.LayerConfig(H, E, k, I, Is, "bf16")
+    good = dict(w_router=(E, H), w_gate=(E, I, H), w_up=(E, I, H), w_down=(E, H, I),
+                ws_gate=(Is, H), ws_up=(Is, H), ws_down=(H, Is))
+
+    def make(**over):
+        ws = {n: _FakeCudaTensor(shape, bf) for n, shape in good.items()}
+        ws.update(over)
+        return smt.MoELayer(cfg, **ws, device=0)
+
+    for name, shape in good.items():
+        wrong = tuple(reversed(shape)) if len(set(shape)) > 1 else shape + (1,)
+        with pytest.raises(ValueError, match=name):
+            make(**{name: _FakeCudaTensor(wrong, bf)})
+        with pytest.raises(ValueError, match=name):
+            make(**{name: _FakeCudaTensor(shape, torch.float32)})
+        with pytest.raises(ValueError, match=name):
+            make(**{name: _FakeCudaTensor(shape, bf, contiguous=False)})
+        with pytest.raises(ValueError, match=name):
+            make(**{name: None})
+    with pytest.raises(ValueError, match="rms_weight"):
+        make(rms_weight=_FakeCudaTensor((H + 1,), bf))
