@@ -58,7 +58,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     extra = ["-Xptxas", "-v"] if verbose else []
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        # objects private to this process, like the library's temporary below
+        obj = os.path.join(BUILD, f"{os.path.basename(src)}.{os.getpid()}.o")
         cmd = [cc, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -74,6 +75,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     tmp = f"{LIB}.{os.getpid()}.tmp"      # private per process; the replace is atomic
     cmd = [cc, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
+    for o in objs:
+        os.remove(o)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stderr}")
     os.replace(tmp, LIB)
