@@ -2,6 +2,8 @@
 import ctypes
 import os
 import re
+import shutil
+import subprocess
 
 import pytest
 
@@ -189,3 +191,52 @@ def test_binding_weight_checks_without_gpu():
             make(**{name: None})
     with pytest.raises(ValueError, match="rms_weight"):
         make(rms_weight=_FakeCudaTensor((H + 1,), bf))
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "moe.h"
+
+static int fails = 0;
+#define CHECK(c) do { if (!(c)) { ++fails; printf("failed: %s (line %d)\n", #c, __LINE__); } } while (0)
+
+int main(void) {
+    CHECK(strstr(moe_version(), "sm_100a") != NULL);
+    CHECK(strcmp(moe_status_string(MOE_OK), "ok") == 0);
+    CHECK(strcmp(moe_status_string((moe_status)42), "unknown status") == 0);
+    moe_handle h = (moe_handle)0;
+    moe_config cfg = {1024, 128, 6, 384, 768, MOE_DTYPE_BF16, 1, 1e-6f};
+    /* argument errors are returned before any CUDA call */
+    CHECK(moe_create(NULL, 0, 0, 0, 0, 0, 0, 0, 0, 0, &h) == MOE_ERR_INVALID_ARG);
+    CHECK(moe_create(&cfg, 0, 0, 0, 0, 0, 0, 0, 0, 0, &h) == MOE_ERR_INVALID_ARG);
+    CHECK(h == NULL);
+    CHECK(strlen(moe_last_error(NULL)) > 0);
+    CHECK(moe_forward(NULL, 0, 0, 0, 8, 0, 0, 0) == MOE_ERR_INVALID_ARG);
+    CHECK(moe_route(NULL, 0, 8, 0, 0, 0) == MOE_ERR_INVALID_ARG);
+    CHECK(moe_reserve(NULL, 8) == MOE_ERR_INVALID_ARG);
+    CHECK(moe_set_option(NULL, MOE_OPT_WAIT_LIMIT_NS, 1) == MOE_ERR_INVALID_ARG);
+    CHECK(moe_kernel_stats(NULL, NULL, NULL, 0) == MOE_ERR_INVALID_ARG);
+    CHECK(moe_destroy(NULL) == MOE_OK);
+    CHECK(moe_route_noalloc(&cfg, 0, 0, 0, 0, 0, 0, 0) == MOE_OK);           /* T = 0 */
+    CHECK(moe_route_noalloc(&cfg, (const void*)8, (const void*)16, 0, 4,
+                            (int32_t*)16, (float*)16, 0) == MOE_ERR_INVALID_ARG);  /* misaligned x */
+    printf(fails ? "FAIL %d\n" : "OK\n", fails);
+    return fails ? 1 : 0;
+}
+"""
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+def test_header_is_c_and_links_from_c(lib, tmp_path):
+    """include/moe.h compiles as C11 and a C program links against the library and gets
+    the documented argument errors (no GPU: nothing here reaches the CUDA runtime)."""
+    src = tmp_path / "abi.c"
+    exe = tmp_path / "abi"
+    src.write_text(C_PROGRAM)
+    libdir = os.path.dirname(smt.LIB_PATH)
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L", libdir, "-lmoe_b200",
+                    f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip().endswith("OK"), r.stdout + r.stderr
