@@ -300,7 +300,10 @@ def test_back_to_back_residual_stream(T):
     no pre-norm, the few-token path with the one-CTA router) give the same bits when
     issued back to back on one stream as with a device synchronisation after every call:
     each call reads x only after the previous call has written it."""
-    inp = synth.make("talker_decode", T=T)
+    # Talker sizes with weights ~ N(0, 0.01): the stream x <- x + MoE(x) stays bounded
+    # over 48 steps (max |x| from about 4.5 to 6 in the oracle's bf16 chain), where the
+    # N(0, 0.02) decode weights overflow after about 20
+    inp = synth.make_custom(1024, 128, 6, 384, 768, T, "bf16", seed=40, w_scale=0.01)
     layer, _ = _layer(inp)
     x0 = smt.to_device(inp.x)
     a, b = x0.clone(), x0.clone()
@@ -311,7 +314,7 @@ def test_back_to_back_residual_stream(T):
         layer.forward(b, residual=b, out=b)
         torch.cuda.synchronize()
     assert layer.check() == 0
-    assert torch.isfinite(a.float()).all()
+    assert torch.isfinite(a.float()).all() and not torch.equal(a, x0)
     assert torch.equal(a, b)
 
 
