@@ -349,6 +349,8 @@ def main():
     import torch
     import torch.distributed as dist
     import sparse_moe_transformer_b200 as smt
+    from sparse_moe_transformer_b200 import build as smt_build
+    smt_build.build()           # no-op when the in-tree library is up to date
 
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
