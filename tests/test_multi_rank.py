@@ -2,7 +2,7 @@
 
 The layer shards as replicas: each rank runs its own copy on its own tokens and
 only the timing is reduced (max over ranks).  Checked here without a GPU:
-distinct per-rank token batches, the max-over-ranks reduction the bench uses,
+the bench's per-rank inputs (one set of weights, distinct token batches), the max-over-ranks reduction the bench uses,
 and that per-rank shards of a batch reproduce the full batch (tokens are
 independent, so replicas need no exchange).
 """
@@ -33,11 +33,13 @@ def _worker(rank, world, port, out):
         import bench
         import oracle
         import synth
-        # per-rank token batches of the decode workload are distinct
-        wl = synth.WORKLOADS["tiny_fp32"]
-        x = synth.make_tokens(wl, 4, seed=rank * 1000)
-        gathered = [torch.zeros(4, wl.H) for _ in range(world)]
+        # the bench's per-rank inputs: the same weights on every rank, distinct tokens
+        wl, copies = bench.build_inputs("tiny_fp32", rank, 1)
+        (layers, x), = copies
+        gathered = [torch.zeros(wl.T, wl.H) for _ in range(world)]
         dist.all_gather(gathered, torch.from_numpy(x.astype(np.float32)))
+        wr = [torch.zeros(wl.E, wl.H) for _ in range(world)]
+        dist.all_gather(wr, torch.from_numpy(layers[0].w_router.astype(np.float32)))
         # the slowest rank sets the time
         t = bench.max_over_ranks(10.0 + rank, dist)
         # shards of one batch, routed on their own rank, equal the full batch
@@ -52,6 +54,7 @@ def _worker(rank, world, port, out):
         if rank == 0:
             y_full, _, _, _ = o.forward(inp.x)
             out.put(dict(distinct=not torch.equal(gathered[0], gathered[1]), t=t,
+                         same_weights=torch.equal(wr[0], wr[1]),
                          same=bool(np.array_equal(torch.cat(parts).numpy(), y_full))))
         dist.barrier()
     finally:
@@ -69,6 +72,6 @@ def test_replicas_two_gloo_ranks():
     for p in procs:
         p.join(timeout=120)
         assert p.exitcode == 0
-    assert res["distinct"]
+    assert res["distinct"] and res["same_weights"]
     assert res["t"] == 11.0
     assert res["same"]
