@@ -77,6 +77,8 @@ SHAPES = [  # H, E, k, I, Is, T   (narrow and wide tile paths, ragged tails, k=1
     (256, 128, 2, 128, 128, 65),      # ... one more token: the CUDA-core router
     (1024, 1, 1, 3072, 0, 8),         # dense SwiGLU FFN as a one-expert layer (1024-3072-1024)
     (1024, 1, 1, 3072, 0, 300),       # ... at prefill size
+    (256, 16, 4, 128, 128, 256),      # few-token kernel at its largest: T k = 1024 slots
+    (256, 16, 4, 128, 128, 257),      # ... one token more: the grouped path
 ]
 
 
