@@ -730,7 +730,11 @@ moe_status moe_last_routing(moe_handle h, int32_t* counts, int32_t* offsets, int
         const int E = h->d.E, k = h->d.k, S = h->last_T * k;
         std::vector<int32_t> idx(S), cnt(E, 0), off(E + 1, 0);
         if (S) CUDA_TRY(cudaMemcpy(idx.data(), h->rb.topk_idx, (size_t)S * 4, cudaMemcpyDeviceToHost));
-        for (int i = 0; i < S; ++i) cnt[idx[i]]++;
+        for (int i = 0; i < S; ++i) {
+            if (idx[i] < 0 || idx[i] >= E)     // only after a failed call: never index with it
+                return fail(MOE_ERR_DEVICE_CHECK, "recorded expert index %d out of range", idx[i]);
+            cnt[idx[i]]++;
+        }
         for (int e = 0; e < E; ++e) off[e + 1] = off[e] + cnt[e];
         if (counts) memcpy(counts, cnt.data(), (size_t)E * 4);
         if (offsets) memcpy(offsets, off.data(), (size_t)(E + 1) * 4);
