@@ -140,6 +140,9 @@ moe_status moe_forward_host(moe_handle h, const void* x_host, const void* residu
  * counts [E]: tokens per expert; offsets [E+1]: exclusive prefix sum of counts
  * (first permuted row of each expert); token_slot [T][k]: permuted row of
  * token t's j-th selected expert, rows of one expert ordered by token index.
+ * Errors: INVALID_ARG (NULL handle, no workspace), CUDA, DEVICE_CHECK (the
+ * recorded routing holds an invalid expert index, possible only after a failed
+ * call).
  */
 moe_status moe_last_routing(moe_handle h, int32_t* counts, int32_t* offsets,
                             int32_t* token_slot, void* stream);
