@@ -91,3 +91,19 @@ def test_router_scale_sharpens_weights(case, c):
     for t in np.nonzero(clear)[0]:
         # w_i / w_0 = exp(l_i - l_0); scaling the logits by c raises the ratio to the c
         assert np.allclose(w_c[t] / w_c[t, 0], (w[t] / w[t, 0]) ** c, rtol=1e-9, atol=0)
+
+
+def test_thread_count_does_not_change_results():
+    """The oracle parallelises over tokens only, so any thread count gives the same bits
+    (the parity tests and the timed baselines use different counts)."""
+    import synth
+    inp = synth.make("talker_decode")
+    L, wl = inp.layers[0], inp.workload
+    o = oracle.Oracle(LayerWeights(**L.arrays(), top_k=wl.k))
+    ref = o.forward(inp.x, nthreads=1)
+    for n in (2, 3, 0):
+        out = o.forward(inp.x, nthreads=n)
+        assert all(np.array_equal(a, b) for a, b in zip(out, ref))
+    r1 = o.route(inp.x, nthreads=1)
+    r0 = o.route(inp.x, nthreads=0)
+    assert all(np.array_equal(a, b) for a, b in zip(r0, r1))
