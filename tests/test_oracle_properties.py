@@ -63,6 +63,8 @@ def test_selection_and_weights(case):
             rest = np.delete(logits[t], idx[t])
             assert sel.min() >= rest.max()                      # a Top-k of the logits
             assert abs(gap[t] - (sel.min() - rest.max())) < 1e-12
+        else:
+            assert gap[t] == np.inf                             # no (k+1)-th expert
 
 
 @SETTINGS
